@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the routed heterogeneous-attention step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl heta|reference]
+
+One step is one pass of the whole path over one sample of the Wan2.1-1.3B
+latent shape (B=1, H=12, d=128, grid 21x30x52, N=32760, rho=0.2, window
+3x9x9): route the previous step's uncertainty u -> routed attention (dense
+rows + windowed local rows, merged) -> uncertainty head on the step's hidden
+states X (C=1536) producing the next step's u.  Inputs are seeded synthetic
+data resident in HBM; Q/K/V/X (402 MB) exceed the 126 MB L2, so no flush is
+needed between steps.
+
+Rank 0 prints one JSON line.  Under torchrun each rank processes its own
+independent sample (weak scaling, no data-path collective); the timed region
+is bracketed by barriers and the elapsed time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (a
+deliberately slow baseline, not a target), on a bounded sample of the same
+workload per step.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from uncertainty_routed_heterogeneous_b200 import dist as D  # noqa: E402
+from uncertainty_routed_heterogeneous_b200 import workloads as W  # noqa: E402
+
+METRIC = "routed-attention tokens/s and TFLOP/s (fraction of B200 bf16 peak) at 1 GPU"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[1])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["heta", "reference"], default="heta")
+    p.add_argument("--workload", default=W.WAN21.name, choices=sorted(W.ALL))
+    p.add_argument("--cpu-tokens", type=int, default=1536,
+                   help="tokens in the oracle's bounded CPU sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-dense-compare", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        pk["source"] = "measured"
+        return pk
+    except (OSError, ValueError):
+        pk = dict(FALLBACK_PEAKS)
+        pk["source"] = "fallback"
+        return pk
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; no setting is changed)
+# ----------------------------------------------------------------------------
+
+
+class ClockSampler:
+    REASONS = {  # NVML clocks-event-reason bits
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, torch_device_index, period_s=0.01):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._on = threading.Event()
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 -- clocks are best-effort metadata
+            self.error = repr(e)
+            return
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            if self._on.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                    self.samples.append((mhz, rs))
+                except Exception:  # noqa: BLE001
+                    pass
+            time.sleep(self.period)
+
+    def start(self):
+        self._on.set()
+
+    def stop(self):
+        self._on.clear()
+
+    def close(self):
+        self._stop.set()
+
+    def summary(self):
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": "NVML unavailable: %s" % getattr(self, "error", "")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = [s[0] for s in self.samples]
+        active = set()
+        for _, rs in self.samples:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    active.add(name)
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(active), "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------
+# CPU side: the fp64 oracle on a bounded sample (reference arm / cpu_baseline)
+# ----------------------------------------------------------------------------
+
+
+class OracleSample:
+    """Host copies of one sample and the oracle calls that make one 'step'."""
+
+    def __init__(self, w, n_tokens, seed=123):
+        import oracle
+        self.oracle = oracle
+        self.w = w
+        q, k, v = W.make_qkv(w)
+        self.q, self.k, self.v = W.bf16_to_f32(q), W.bf16_to_f32(k), W.bf16_to_f32(v)
+        self.u = W.make_u(w)
+        X, self.wv = W.make_head(w)
+        self.X = W.bf16_to_f32(X)
+        self.kk = oracle.dense_count(w.N, w.rho)
+        self.n_tokens = min(n_tokens, w.N)
+        self.rng = np.random.default_rng(seed)
+
+    def step(self):
+        """Routes the whole sample, then attention + head for a token sample."""
+        o, w = self.oracle, self.w
+        dense, _, _ = o.route(self.u[:1], self.kk)
+        toks = self.rng.choice(w.N, size=self.n_tokens, replace=False)
+        rows = (np.arange(w.H)[:, None] * w.N + toks[None, :]).ravel().astype(np.int64)
+        o.attention_rows(self.q[:1], self.k[:1], self.v[:1], w.grid, w.win, dense, rows)
+        o.uncertainty(self.X[:1, toks], self.wv)
+        return self.n_tokens
+
+    def describe(self):
+        return ("%d of %d tokens of one sample (random), all %d heads, at the workload's own "
+                "dense/local mix; routing over the full sample; head on the sampled tokens"
+                % (self.n_tokens, self.w.N, self.w.H))
+
+
+def run_reference(args, info):
+    import oracle
+    if info.rank != 0:
+        return 0
+    w = W.ALL[args.workload]
+    s = OracleSample(w, n_tokens=max(16, args.cpu_tokens // 6))
+    for _ in range(args.warmup):
+        s.step()
+    t0 = time.perf_counter()
+    toks = 0
+    for _ in range(args.steps):
+        toks += s.step()
+    dt = time.perf_counter() - t0
+    value = toks / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": s.describe()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def cpu_baseline(args, w):
+    import oracle
+    s = OracleSample(w, n_tokens=args.cpu_tokens)
+    s.step()  # warm: page in, build
+    t0 = time.perf_counter()
+    n = s.step()
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": s.describe(), "seconds": dt}
+
+
+def config_of(w, n_gpus):
+    k = math.ceil(round(w.rho * w.N, 9))
+    return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d,
+            "grid": "x".join(map(str, w.grid)), "N": w.N, "window": "x".join(map(str, w.win)),
+            "rho": w.rho, "k": k, "head_C": w.C, "u": w.u_kind,
+            "l2": "inputs larger than L2 (Q/K/V/X %.0f MB per step)" % (
+                (3 * w.B * w.H * w.N * w.d * 2 + w.B * w.N * w.C * 2) / 1e6),
+            "parallelism": "dp%d: one independent sample per GPU" % n_gpus}
+
+
+# ----------------------------------------------------------------------------
+# GPU arm
+# ----------------------------------------------------------------------------
+
+
+def run_heta(args, info):
+    import torch
+
+    import uncertainty_routed_heterogeneous_b200 as heta
+
+    torch.cuda.set_device(info.local_rank)
+    dev = torch.device("cuda", info.local_rank)
+    D.init("nccl", info, timeout_s=300)
+    heta.load()
+    base = W.ALL[args.workload]
+    w = D.rank_workload(base, info.rank)
+
+    # ---- inputs: host (pinned) and resident device copies -------------------
+    def pinned_bf16(bits):
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory()
+
+    q, k, v = W.make_qkv(w)
+    X, wv = W.make_head(w)
+    u = W.make_u(w)
+    h_Q, h_K, h_V, h_X = (pinned_bf16(a) for a in (q, k, v, X))
+    del q, k, v, X
+    h_u = torch.from_numpy(u).pin_memory()
+    h_w = torch.from_numpy(wv)
+    d_Q, d_K, d_V, d_X = (t.to(dev) for t in (h_Q, h_K, h_V, h_X))
+    d_u = h_u.to(dev)
+    d_w = h_w.to(dev)
+    kk = heta.dense_count(w.N, w.rho)
+    dense = torch.empty((w.B, kk), dtype=torch.int32, device=dev)
+    local = torch.empty((w.B, w.N - kk), dtype=torch.int32, device=dev)
+    out = torch.empty_like(d_Q)
+    u_next = torch.empty((w.B, w.N), dtype=torch.float32, device=dev)
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    h_unext = torch.empty(u_next.shape, dtype=torch.float32).pin_memory()
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record()
+        heta.route(d_u, kk, out=(dense, local, None, None))
+        if ev is not None:
+            ev[1].record()
+        heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense, out=out)
+        if ev is not None:
+            ev[2].record()
+        heta.uncertainty(d_X, d_w, 0.0, out=u_next)
+        if ev is not None:
+            ev[3].record()
+
+    launches_per_step = 1 + (1 if kk > 0 else 0) + (1 if kk < w.N else 0) + 1
+    flops = heta.attention_flops(w.B, w.H, w.d, w.N, kk, w.M)
+
+    sampler = ClockSampler(info.local_rank)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    D.barrier(info, dev)
+    torch.cuda.synchronize()
+    sampler.start()
+    t_start.record()
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    sampler.stop()
+    D.barrier(info, dev)
+    ms_local = t_start.elapsed_time(t_end)
+    ms_total = D.max_over_ranks(ms_local, info, dev)
+    route_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    head_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    tokens_per_step = w.B * w.N * info.world
+    value = tokens_per_step * args.steps / (ms_total / 1e3)
+
+    # ---- our own full dense attention (rho = 1) at the same shape -----------
+    dense_cmp = None
+    if not args.no_dense_compare:
+        all_idx = torch.arange(w.N, dtype=torch.int32, device=dev).repeat(w.B, 1).contiguous()
+        heta.attention(d_Q, d_K, d_V, w.grid, w.win, all_idx, out=out)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 3
+        e0.record()
+        for _ in range(reps):
+            heta.attention(d_Q, d_K, d_V, w.grid, w.win, all_idx, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+        full_ms = e0.elapsed_time(e1) / reps
+        full_flops = heta.attention_flops(w.B, w.H, w.d, w.N, w.N, w.M)
+        dense_cmp = {"ms": full_ms, "tflops": full_flops / (full_ms * 1e9),
+                     "speedup_of_routed": full_ms / attn_ms}
+
+    # ---- end to end through the public API with host buffers ----------------
+    e2e = None
+    if not args.no_e2e:
+        ke = max(1, min(args.steps, 10))
+
+        def e2e_step():
+            d_Q.copy_(h_Q, non_blocking=True)
+            d_K.copy_(h_K, non_blocking=True)
+            d_V.copy_(h_V, non_blocking=True)
+            d_X.copy_(h_X, non_blocking=True)
+            d_u.copy_(h_u, non_blocking=True)
+            step()
+            h_out.copy_(out, non_blocking=True)
+            h_unext.copy_(u_next, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        D.barrier(info, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(ke):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = D.max_over_ranks(e0.elapsed_time(e1), info, dev)
+        h2d = sum(t.numel() * t.element_size() for t in (h_Q, h_K, h_V, h_X, h_u))
+        d2h = sum(t.numel() * t.element_size() for t in (h_out, h_unext))
+        e2e = {"value": tokens_per_step * ke / (e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
+
+    cpu = None
+    if info.rank == 0 and info.world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args, base)
+
+    sampler.close()
+    if info.rank != 0:
+        return 0
+    peaks = load_peaks()
+    tflops = flops / (attn_ms * 1e9)
+    peak = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; Wan2.1-1.3B latent shape; no model weights)",
+        "config": config_of(base, info.world),
+        "attention_tflops": tflops,
+        "kernel_ms": {"route": route_ms, "attention": attn_ms, "head": head_ms},
+        "roofline": {"bound": "tensor", "kernel": "heta_attention (dense + local kernels)",
+                     "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "frac_of_burst": tflops / peaks["bf16_tflops"],
+                     "peak_source": "%s sustained bf16 (cuBLAS)" % peaks["source"],
+                     "traffic": None, "algorithmic_flops": flops},
+        "head_roofline": {"bound": "hbm",
+                          "achieved": (w.B * w.N * w.C * 2 + w.C * 4 + w.B * w.N * 4) /
+                          (head_ms * 1e6),
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+        "dense_compare": dense_cmp,
+        "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "cpu_baseline": cpu, "clocks": sampler.summary(),
+    }
+    line["head_roofline"]["frac"] = line["head_roofline"]["achieved"] / peaks["hbm_gbs"]
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    info = D.rank_info()
+    if args.impl == "reference":
+        return run_reference(args, info)
+    rc = run_heta(args, info)
+    if info.world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return rc
+
+
+if __name__ == "__main__":
+    sys.exit(main())

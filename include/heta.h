@@ -1,0 +1,149 @@
+/*
+ * heta.h -- C ABI of libheta, the B200 (sm_100a) heterogeneous-attention path.
+ *
+ * The method: "Where Compute Matters: Heterogeneous Attention for Efficient
+ * Video Diffusion" (HetA-DiT).  A per-token uncertainty u (Eq. (7)) from the
+ * previous denoising step picks, per sample, the tokens whose queries get
+ * dense attention over all N keys (Eq. (2)); every other token attends over a
+ * 3D spatio-temporal window of the latent grid (Eq. (3)); the two results are
+ * merged row by row into one output (Eq. (13)).  The routing rule of
+ * Eq. (11)-(12) is taken in top-k form: exactly k = ceil(rho*N) tokens per
+ * sample go dense, rho being the dense fraction of Eq. (14).
+ *
+ * Conventions shared by every entry point
+ *   - Every array pointer is a DEVICE pointer owned by the caller.  The
+ *     library never allocates, frees or retains device memory; it holds no
+ *     state between calls and is safe to call from several host threads.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream).  Calls return before the GPU
+ *     finishes.
+ *   - Argument errors are detected on the host and returned synchronously
+ *     (HETA_ERR_INVALID_ARG / HETA_ERR_UNSUPPORTED) with nothing launched.
+ *     A failed launch returns HETA_ERR_CUDA.
+ *   - Conditions only the GPU can see (a NaN in u) are reported through the
+ *     optional `status_dev` (device int32, may be NULL): a kernel that detects
+ *     one raises it to that code with an atomic max.  The library never
+ *     clears it; zero it before the call and read it after synchronising.
+ *   - bf16 tensors are passed as uint16_t bit patterns (round-to-nearest-even
+ *     values), fp32 as float.  All pointers must be 16-byte aligned.
+ *   - Token order inside a sample is i = (t*Hg + h)*Wg + w on a latent grid
+ *     of Tg x Hg x Wg = N tokens.
+ */
+#ifndef HETA_H
+#define HETA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HETA_API __attribute__((visibility("default")))
+#else
+#define HETA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HETA_OK = 0,
+    HETA_ERR_INVALID_ARG = 1,  /* bad size, pointer, alignment or value     */
+    HETA_ERR_UNSUPPORTED = 2,  /* valid, but outside what the kernels cover */
+    HETA_ERR_CUDA = 3,         /* a CUDA launch or driver call failed       */
+    HETA_ERR_NONFINITE = 4,    /* NaN seen in u (reported via status_dev)   */
+    HETA_ERR_TIMEOUT = 5       /* a bounded wait inside a kernel ran out    */
+} heta_status;
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+HETA_API const char *heta_status_string(int status);
+
+/* Library ABI version: (major << 16) | minor. */
+HETA_API int heta_version(void);
+
+/*
+ * Dense tokens per sample: *k_out = ceil(rho * N).
+ *
+ * rho is the dense-query fraction of Eq. (14).  It is read as the decimal
+ * fraction the caller states: when the IEEE product rho*N lies within 1e-12
+ * (relative) of an integer, that integer is used, so rho = 0.1, N = 30 gives
+ * 3.  Requires N >= 0 and 0 <= rho <= 1; otherwise HETA_ERR_INVALID_ARG.
+ * Host-only; touches no device.
+ */
+HETA_API heta_status heta_dense_count(int N, double rho, int *k_out);
+
+/*
+ * heta_route -- per-sample top-k selection and compaction (Eq. (11)-(12)).
+ *
+ * For each sample b the k tokens with the largest u[b,:] form the dense set
+ * D_b.  Ties at the threshold are taken in increasing token index; -0.0 and
+ * +0.0 compare equal; +-inf are ordinary values.  A NaN anywhere in u raises
+ * status_dev to HETA_ERR_NONFINITE (outputs are then unspecified).
+ *
+ *   u          [B,N] fp32, read only.
+ *   dense_idx  [B,k] int32 out: D_b in increasing token order.
+ *   local_idx  [B,N-k] int32 out: the complement, increasing.
+ *   thresh_out [B] fp32 out, or NULL: the k-th largest u of each sample
+ *              (the effective threshold T of Eq. (11)); +inf when k == 0.
+ *   mask_out   [B,N] uint8 out, or NULL: the paper's m_i, 1 = local, 0 = dense.
+ *   status_dev device int32, or NULL (see conventions).
+ *
+ * Requires B >= 1, 1 <= N <= 53248 (one sample's keys live in one SM's
+ * shared memory), 0 <= k <= N, B*N < 2^31.  One CTA per sample.
+ */
+HETA_API heta_status heta_route(const float *u, int B, int N, int k,
+                       int32_t *dense_idx, int32_t *local_idx,
+                       float *thresh_out, uint8_t *mask_out,
+                       int32_t *status_dev, void *stream);
+
+/*
+ * heta_attention -- routed heterogeneous self-attention (Eq. (2), (3), (13)).
+ *
+ * For every sample b, head h and token i:
+ *   i in D_b : out[b,h,i] = sum_j softmax_j(scale * q_i.k_j) v_j over all N
+ *              keys (Eq. (2));
+ *   otherwise: the same softmax restricted to the window N(i) (Eq. (3)): the
+ *              box [s_t, s_t+wt) x [s_h, s_h+wh) x [s_w, s_w+ww) with
+ *              s_a = clamp(a - floor(w_a/2), 0, extent_a - w_a), so every
+ *              window holds exactly wt*wh*ww keys.
+ * Keys and values are always all N tokens of (b,h); only queries are routed.
+ *
+ *   Q, K, V    [B,H,N,d] bf16, contiguous, read only.
+ *   dense_idx  [B,k] int32: D_b, strictly increasing, 0 <= idx < N (the
+ *              heta_route output).  Not checked on the device: indices out
+ *              of range or out of order give unspecified rows.
+ *   out        [B,H,N,d] bf16 out; every row is written exactly once.
+ *   scale      softmax scale, normally 1/sqrt(d).
+ *
+ * Requires d in {64, 128}; odd wt, wh, ww with 1 <= w_a <= extent_a;
+ * N = Tg*Hg*Wg; 0 <= k <= N; B*H*N*d < 2^40.  Other d or even windows give
+ * HETA_ERR_UNSUPPORTED.
+ */
+HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
+                           const uint16_t *V, int B, int H, int d,
+                           int Tg, int Hg, int Wg, int wt, int wh, int ww,
+                           float scale, const int32_t *dense_idx, int k,
+                           uint16_t *out, int32_t *status_dev, void *stream);
+
+/*
+ * heta_uncertainty -- the lightweight per-token uncertainty head (Eq. (7)).
+ *
+ * u_out[b,i] = softplus(sum_c X[b,i,c] * w[c] + bias), softplus(z) =
+ * log(1 + e^z), so u >= 0 as Eq. (7) requires.  The paper gives no
+ * architecture beyond "lightweight"; a linear map to one scalar followed by
+ * softplus is the form used here.  fp32 accumulation.
+ *
+ *   X      [B,N,C] bf16 (the final hidden states of the step), read only.
+ *   w      [C] fp32; bias a host scalar.
+ *   u_out  [B,N] fp32 out: the u that routes the next denoising step.
+ *
+ * Requires B, N >= 1, C a multiple of 8 with 8 <= C <= 16384.
+ */
+HETA_API heta_status heta_uncertainty(const uint16_t *X, const float *w, float bias,
+                             int B, int N, int C, float *u_out,
+                             int32_t *status_dev, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HETA_H */

@@ -1,0 +1,109 @@
+"""The C-ABI library builds, loads and exports what include/heta.h declares.
+
+CPU only: no call here reaches the GPU.  The validation cases return from the
+host-side checks before any CUDA call is made.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import uncertainty_routed_heterogeneous_b200 as heta
+from uncertainty_routed_heterogeneous_b200 import build as heta_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    heta_build.build()
+    return heta.load()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"HETA_API\s+[\w\s\*]*?\b(heta_\w+)\s*\(", text))
+    return names
+
+
+def test_header_declares_the_three_path_calls():
+    names = declared_symbols()
+    assert {"heta_route", "heta_attention", "heta_uncertainty", "heta_dense_count",
+            "heta_status_string", "heta_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        s = heta.status_string(code)
+        assert s and s != "unknown status"
+    assert heta.status_string(99) == "unknown status"
+    assert lib.heta_version() >> 16 == 1
+
+
+def test_dense_count_matches_oracle(lib):
+    for N in (0, 1, 7, 10, 30, 100, 256, 27280, 32760):
+        for rho in (0.0, 0.01, 0.05, 0.07, 0.1, 0.2, 0.25, 0.3, 0.35, 0.5, 0.99, 1.0):
+            assert heta.dense_count(N, rho) == oracle.dense_count(N, rho), (N, rho)
+    with pytest.raises(heta.HetaError):
+        heta.dense_count(10, 1.5)
+    with pytest.raises(heta.HetaError):
+        heta.dense_count(-1, 0.5)
+
+
+def test_host_validation_returns_before_any_launch(lib):
+    N = None
+    # B = 0 / k > N / null pointers are rejected on the host
+    assert lib.heta_route(N, 0, 10, 1, N, N, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    assert lib.heta_route(N, 1, 10, 11, N, N, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    assert lib.heta_route(N, 1, 10, 2, N, N, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.heta_route(fake, 1, 60000, 2, fake, fake, N, N, N, N) == \
+        heta.HETA_ERR_UNSUPPORTED
+    # misaligned pointer
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert lib.heta_route(odd, 1, 10, 2, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    args = [fake, fake, fake, 1, 2, 128, 4, 8, 8, 3, 3, 3, ctypes.c_float(0.1), fake, 3, fake, N, N]
+    bad_d = list(args)
+    bad_d[5] = 96
+    assert lib.heta_attention(*bad_d) == heta.HETA_ERR_UNSUPPORTED
+    even_win = list(args)
+    even_win[10] = 4
+    assert lib.heta_attention(*even_win) == heta.HETA_ERR_UNSUPPORTED
+    big_win = list(args)
+    big_win[9] = 5
+    assert lib.heta_attention(*big_win) == heta.HETA_ERR_INVALID_ARG
+    bad_k = list(args)
+    bad_k[14] = 257
+    assert lib.heta_attention(*bad_k) == heta.HETA_ERR_INVALID_ARG
+    bad_scale = list(args)
+    bad_scale[12] = ctypes.c_float(float("nan"))
+    assert lib.heta_attention(*bad_scale) == heta.HETA_ERR_INVALID_ARG
+    assert lib.heta_uncertainty(fake, fake, ctypes.c_float(0.0), 1, 10, 12, fake, N, N) == \
+        heta.HETA_ERR_INVALID_ARG
+    assert lib.heta_uncertainty(fake, fake, ctypes.c_float(0.0), 1, 10, 32768, fake, N, N) == \
+        heta.HETA_ERR_UNSUPPORTED
+
+
+def test_flop_model_matches_the_papers_reduction():
+    """Eq. (14) at the Wan2.1-1.3B latent shape, rho = 0.2, 3x9x9 window.
+
+    The dense/heterogeneous FLOP ratio comes out at 4.856; Table 5 prints an
+    attention-FLOPs reduction of 4.87x for Wan2.1-1.3B.  Context only: the
+    paper does not state which window produced its table.
+    """
+    N, M = 32760, 243
+    k = heta.dense_count(N, 0.2)
+    full = heta.attention_flops(1, 12, 128, N, N, M)
+    het = heta.attention_flops(1, 12, 128, N, k, M)
+    assert abs(full / het - 4.87) < 0.02
+    assert het == 4 * 128 * 12 * (k * N + (N - k) * M)

@@ -1,0 +1,55 @@
+"""Multi-rank host logic on CPU: gloo, world size 2, two real processes."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+from uncertainty_routed_heterogeneous_b200 import dist as D
+from uncertainty_routed_heterogeneous_b200 import workloads as W
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    info = D.rank_info()
+    D.init("gloo", info, timeout_s=30)
+    D.barrier(info)
+    # each rank reports its own elapsed time; every rank must see the max
+    m = D.max_over_ranks(1.5 + rank, info)
+    w = D.rank_workload(W.WAN21, info.rank)
+    q.put((rank, m, w.qkv_seed, w.u_seeds, w.x_seed, D.head_range(12, world, rank)))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_two_ranks_agree_on_max_and_get_independent_samples():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    (r0, m0, s0, u0, x0, h0), (r1, m1, s1, u1, x1, h1) = res
+    assert m0 == m1 == 2.5
+    assert s0 != s1 and u0 != u1 and x0 != x1
+    assert h0 == (0, 6) and h1 == (6, 12)
+
+
+@pytest.mark.parametrize("H,world", [(12, 1), (12, 5), (24, 8), (3, 4)])
+def test_head_ranges_partition(H, world):
+    seen = []
+    for r in range(world):
+        lo, hi = D.head_range(H, world, r)
+        seen += list(range(lo, hi))
+    assert seen == list(range(H))

@@ -1,0 +1,92 @@
+"""heta_route on the GPU against the oracle: index lists must be bit-exact.
+
+"Where Compute Matters: Heterogeneous Attention for Efficient Video
+Diffusion", §3.2.2 Eq. (11)-(12), in top-k form (k = ceil(rho*N) per sample,
+Eq. (14)); ties go to the smaller token index.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from helpers import to_dev
+from test_oracle_pins import read_route_ties
+from uncertainty_routed_heterogeneous_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def check_route(heta, u, k):
+    import torch
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    d, l, th, m = heta.route(to_dev(u), k, want_thresh=True, want_mask=True, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    od, ol, om = oracle.route(u, k)
+    assert np.array_equal(d.cpu().numpy(), od)
+    assert np.array_equal(l.cpu().numpy(), ol)
+    assert np.array_equal(m.cpu().numpy(), om)
+    th = th.cpu().numpy()
+    for b in range(u.shape[0]):
+        if k == 0:
+            assert th[b] == np.inf
+        else:
+            assert th[b] == u[b, od[b]].min()
+
+
+@pytest.mark.parametrize("name", ["tiny-4x8x8", "wan2.1-1.3b-21x30x52", "wan2.2-5b-31x22x40",
+                                  "wan2.1-1.3b-batched-b2"])
+def test_route_workloads(gpu_lib, name):
+    w = W.ALL[name]
+    u = W.make_u(w)
+    check_route(gpu_lib, u, gpu_lib.dense_count(w.N, w.rho))
+
+
+@pytest.mark.parametrize("kind", ["uniform", "clustered"])
+@pytest.mark.parametrize("rho", W.SWEEP_RHOS)
+def test_route_sweep(gpu_lib, kind, rho):
+    w = W.sweep(rho, kind)
+    check_route(gpu_lib, W.make_u(w), gpu_lib.dense_count(w.N, rho))
+
+
+@pytest.mark.parametrize("case", read_route_ties())
+def test_route_golden_ties(gpu_lib, case):
+    k, u, _, _ = case
+    check_route(gpu_lib, u[None, :].copy(), k)
+
+
+@pytest.mark.parametrize("k", [0, 1, 2, 6551, 32759, 32760])
+def test_route_extreme_k(gpu_lib, k):
+    u = W.make_u(W.WAN21)
+    check_route(gpu_lib, u, k)
+
+
+@pytest.mark.parametrize("N,B,kind", [(1, 1, "u"), (33, 2, "u"), (1001, 3, "u"),
+                                      (53248, 1, "ties"), (32760, 2, "equal"),
+                                      (4097, 2, "signed_zero"), (5000, 1, "denormal"),
+                                      (1024, 4, "inf")])
+def test_route_edge_inputs(gpu_lib, N, B, kind):
+    rng = np.random.default_rng(N * 7 + B)
+    if kind == "u":
+        u = rng.random((B, N), dtype=np.float32)
+    elif kind == "ties":
+        u = rng.integers(0, 7, (B, N)).astype(np.float32)
+    elif kind == "equal":
+        u = np.full((B, N), 0.5, np.float32)
+    elif kind == "signed_zero":
+        u = rng.choice(np.array([-0.0, 0.0, 1.0, -1.0], np.float32), (B, N))
+    elif kind == "denormal":
+        u = (rng.integers(-20, 20, (B, N)) * np.float32(1e-45)).astype(np.float32)
+    else:
+        u = rng.choice(np.array([np.inf, -np.inf, 0.0, 3.0], np.float32), (B, N))
+    for rho in (0.0, 0.2, 0.5, 1.0):
+        check_route(gpu_lib, u, gpu_lib.dense_count(N, rho))
+
+
+def test_route_nan_sets_status(gpu_lib):
+    import torch
+    u = np.random.default_rng(0).random((2, 1000), dtype=np.float32)
+    u[1, 17] = np.nan
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gpu_lib.route(to_dev(u), 100, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == gpu_lib.HETA_ERR_NONFINITE

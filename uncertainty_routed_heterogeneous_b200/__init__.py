@@ -1,0 +1,193 @@
+"""B200-native heterogeneous (uncertainty-routed) attention.
+
+Python binding over the C ABI of ``libheta.so`` (``include/heta.h``).  This
+module only marshals arguments: it checks tensor placement, dtype and shape,
+passes raw device pointers and the current CUDA stream, and turns status codes
+into exceptions.  Every step of the path runs in the library's CUDA kernels;
+there is no CPU or PyTorch fallback -- if the library is missing, every call
+raises.
+
+The method is HetA-DiT ("Where Compute Matters: Heterogeneous Attention for
+Efficient Video Diffusion"): per-sample routing of the most uncertain tokens
+(Eq. (11)-(12), top-k form) to dense attention (Eq. (2)), windowed 3D local
+attention for the rest (Eq. (3)), merged row by row (Eq. (13)); the
+uncertainty head (Eq. (7)) produces the next step's scores.
+"""
+import ctypes
+import math
+import os
+
+__all__ = ["load", "HetaError", "dense_count", "route", "attention", "uncertainty",
+           "status_string", "attention_flops", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libheta.so")
+
+HETA_OK = 0
+HETA_ERR_INVALID_ARG = 1
+HETA_ERR_UNSUPPORTED = 2
+HETA_ERR_CUDA = 3
+HETA_ERR_NONFINITE = 4
+HETA_ERR_TIMEOUT = 5
+
+_lib = None
+
+
+class HetaError(RuntimeError):
+    def __init__(self, code, what=""):
+        self.code = int(code)
+        super().__init__("%s: heta status %d (%s)" % (what, self.code, status_string(self.code)))
+
+
+def load():
+    """Loads libheta.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            "libheta.so is not built (%s). Build it with "
+            "`python -m uncertainty_routed_heterogeneous_b200.build`; "
+            "there is no fallback path." % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, d = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double
+    lib.heta_status_string.argtypes = [i]
+    lib.heta_status_string.restype = ctypes.c_char_p
+    lib.heta_version.argtypes = []
+    lib.heta_version.restype = i
+    lib.heta_dense_count.argtypes = [i, d, ctypes.POINTER(ctypes.c_int)]
+    lib.heta_dense_count.restype = i
+    lib.heta_route.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp]
+    lib.heta_route.restype = i
+    lib.heta_attention.argtypes = [vp, vp, vp] + [i] * 9 + [f, vp, i, vp, vp, vp]
+    lib.heta_attention.restype = i
+    lib.heta_uncertainty.argtypes = [vp, vp, f, i, i, i, vp, vp, vp]
+    lib.heta_uncertainty.restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return load().heta_status_string(int(code)).decode()
+    except RuntimeError:
+        return "library not loaded"
+
+
+def _check(rc, what):
+    if rc != HETA_OK:
+        raise HetaError(rc, what)
+
+
+def _stream():
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t, dtype, name, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError("%s must have %d dims, got %d" % (name, ndim, t.dim()))
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _opt(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def dense_count(N: int, rho: float) -> int:
+    """k = ceil(rho*N) for the decimal rho stated (the dense fraction of Eq. (14))."""
+    k = ctypes.c_int(0)
+    _check(load().heta_dense_count(int(N), float(rho), ctypes.byref(k)), "heta_dense_count")
+    return int(k.value)
+
+
+def route(u, k: int, *, out=None, want_thresh=False, want_mask=False, status=None):
+    """Per-sample top-k routing on the GPU (``heta_route``).
+
+    u: [B,N] float32 CUDA.  Returns (dense_idx [B,k] int32, local_idx [B,N-k]
+    int32, thresh [B] float32 or None, mask [B,N] uint8 or None).
+    ``out`` may pass preallocated (dense_idx, local_idx, thresh, mask).
+    """
+    import torch
+    pu = _dev(u, torch.float32, "u", 2)
+    B, N = u.shape
+    if out is None:
+        dense = torch.empty((B, k), dtype=torch.int32, device=u.device)
+        local = torch.empty((B, N - k), dtype=torch.int32, device=u.device)
+        thresh = torch.empty(B, dtype=torch.float32, device=u.device) if want_thresh else None
+        mask = torch.empty((B, N), dtype=torch.uint8, device=u.device) if want_mask else None
+    else:
+        dense, local, thresh, mask = out
+    rc = load().heta_route(pu, B, N, int(k), _opt(dense) if k > 0 else None,
+                           _opt(local) if k < N else None, _opt(thresh), _opt(mask),
+                           _opt(status), _stream())
+    _check(rc, "heta_route")
+    return dense, local, thresh, mask
+
+
+def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=None):
+    """Routed heterogeneous attention (``heta_attention``).
+
+    Q, K, V: [B,H,N,d] bfloat16 CUDA; grid = (Tg, Hg, Wg) with N = Tg*Hg*Wg;
+    win = (wt, wh, ww) odd; dense_idx: [B,k] int32 CUDA, increasing.
+    Returns out [B,H,N,d] bfloat16.
+    """
+    import torch
+    pq = _dev(Q, torch.bfloat16, "Q", 4)
+    pk = _dev(K, torch.bfloat16, "K", 4)
+    pv = _dev(V, torch.bfloat16, "V", 4)
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V shapes differ")
+    B, H, N, d = Q.shape
+    Tg, Hg, Wg = grid
+    if Tg * Hg * Wg != N:
+        raise ValueError("grid %s does not hold N=%d tokens" % (grid, N))
+    pd = _dev(dense_idx, torch.int32, "dense_idx", 2)
+    if dense_idx.shape[0] != B:
+        raise ValueError("dense_idx batch mismatch")
+    k = dense_idx.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    po = _dev(out, torch.bfloat16, "out", 4)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = load().heta_attention(pq, pk, pv, B, H, d, Tg, Hg, Wg, win[0], win[1], win[2],
+                               float(scale), pd if k > 0 else None, k, po, _opt(status),
+                               _stream())
+    _check(rc, "heta_attention")
+    return out
+
+
+def uncertainty(X, w, bias: float = 0.0, *, out=None, status=None):
+    """u = softplus(X.w + b) per token (``heta_uncertainty``).
+
+    X: [B,N,C] bfloat16 CUDA; w: [C] float32 CUDA.  Returns u [B,N] float32.
+    """
+    import torch
+    px = _dev(X, torch.bfloat16, "X", 3)
+    pw = _dev(w, torch.float32, "w", 1)
+    B, N, C = X.shape
+    if w.shape[0] != C:
+        raise ValueError("w has %d entries, X has C=%d" % (w.shape[0], C))
+    if out is None:
+        out = torch.empty((B, N), dtype=torch.float32, device=X.device)
+    pu = _dev(out, torch.float32, "u_out", 2)
+    rc = load().heta_uncertainty(px, pw, float(bias), B, N, C, pu, _opt(status), _stream())
+    _check(rc, "heta_uncertainty")
+    return out
+
+
+def attention_flops(B: int, H: int, d: int, N: int, k: int, M: int) -> int:
+    """Algorithmic FLOPs of one routed-attention call.
+
+    Two matrix products (q.k and p.v) of 2*d FLOPs per (query, key) pair:
+    k*N pairs for the dense rows and (N-k)*M for the local rows per (b, h) --
+    the two terms of the cost model of Eq. (14).
+    """
+    return 4 * d * H * B * (k * N + (N - k) * M)

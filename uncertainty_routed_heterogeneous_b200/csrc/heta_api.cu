@@ -1,0 +1,101 @@
+// heta_api.cu -- the extern "C" entry points of libheta (declared in heta.h):
+// host-side argument checks, then one asynchronous launch sequence each.
+#include <math.h>
+
+#include "heta_internal.cuh"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+heta_status from_cuda(cudaError_t e) { return e == cudaSuccess ? HETA_OK : HETA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *heta_status_string(int status)
+{
+    switch (status) {
+    case HETA_OK: return "ok";
+    case HETA_ERR_INVALID_ARG: return "invalid argument";
+    case HETA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HETA_ERR_CUDA: return "CUDA error";
+    case HETA_ERR_NONFINITE: return "non-finite (NaN) uncertainty value";
+    case HETA_ERR_TIMEOUT: return "bounded wait in a kernel timed out";
+    default: return "unknown status";
+    }
+}
+
+int heta_version(void) { return (1 << 16) | 0; }
+
+heta_status heta_dense_count(int N, double rho, int *k_out)
+{
+    if (!k_out || N < 0 || !(rho >= 0.0 && rho <= 1.0)) return HETA_ERR_INVALID_ARG;
+    const double prod = rho * (double)N;
+    const double nearest = nearbyint(prod);
+    const double tol = 1e-12 * (prod > 1.0 ? prod : 1.0);
+    int k = fabs(prod - nearest) <= tol ? (int)nearest : (int)ceil(prod);
+    *k_out = k > N ? N : k;
+    return HETA_OK;
+}
+
+heta_status heta_route(const float *u, int B, int N, int k, int32_t *dense_idx,
+                       int32_t *local_idx, float *thresh_out, uint8_t *mask_out,
+                       int32_t *status_dev, void *stream)
+{
+    if (B < 1 || N < 1 || k < 0 || k > N) return HETA_ERR_INVALID_ARG;
+    if ((int64_t)B * N >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
+    if (N > heta::kRouteMaxN) return HETA_ERR_UNSUPPORTED;
+    if (!u || (k > 0 && !dense_idx) || (k < N && !local_idx)) return HETA_ERR_INVALID_ARG;
+    if (!aligned16(u) || (dense_idx && !aligned16(dense_idx)) ||
+        (local_idx && !aligned16(local_idx)) || (thresh_out && !aligned16(thresh_out)) ||
+        (mask_out && !aligned16(mask_out)))
+        return HETA_ERR_INVALID_ARG;
+    return from_cuda(heta::launch_route(u, B, N, k, dense_idx, local_idx, thresh_out,
+                                        mask_out, status_dev,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+heta_status heta_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B,
+                           int H, int d, int Tg, int Hg, int Wg, int wt, int wh, int ww,
+                           float scale, const int32_t *dense_idx, int k, uint16_t *out,
+                           int32_t *status_dev, void *stream)
+{
+    if (B < 1 || H < 1 || Tg < 1 || Hg < 1 || Wg < 1) return HETA_ERR_INVALID_ARG;
+    const int64_t N64 = (int64_t)Tg * Hg * Wg;
+    if (N64 >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
+    const int N = (int)N64;
+    if (k < 0 || k > N) return HETA_ERR_INVALID_ARG;
+    if (wt < 1 || wh < 1 || ww < 1 || wt > Tg || wh > Hg || ww > Wg) return HETA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !isfinite(scale)) return HETA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !out || (k > 0 && !dense_idx)) return HETA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
+        (dense_idx && !aligned16(dense_idx)))
+        return HETA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return HETA_ERR_UNSUPPORTED;
+    if ((wt % 2) == 0 || (wh % 2) == 0 || (ww % 2) == 0) return HETA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H * N * d >= (int64_t)1 << 40) return HETA_ERR_UNSUPPORTED;
+    heta::AttnArgs a;
+    a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
+    a.B = B; a.H = H; a.d = d; a.N = N; a.k = k;
+    a.Tg = Tg; a.Hg = Hg; a.Wg = Wg; a.wt = wt; a.wh = wh; a.ww = ww;
+    a.scale = scale;
+    return from_cuda(heta::launch_attention(a, static_cast<cudaStream_t>(stream)));
+}
+
+heta_status heta_uncertainty(const uint16_t *X, const float *w, float bias, int B, int N,
+                             int C, float *u_out, int32_t *status_dev, void *stream)
+{
+    (void)status_dev;  // the head has no device-detected conditions
+    if (B < 1 || N < 1 || C < 8 || (C % 8) != 0) return HETA_ERR_INVALID_ARG;
+    if (C > 16384) return HETA_ERR_UNSUPPORTED;
+    if ((int64_t)B * N >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
+    if (!X || !w || !u_out) return HETA_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(w) || !aligned16(u_out)) return HETA_ERR_INVALID_ARG;
+    if (!isfinite(bias)) return HETA_ERR_INVALID_ARG;
+    return from_cuda(heta::launch_uncertainty(X, w, bias, B, N, C, u_out,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

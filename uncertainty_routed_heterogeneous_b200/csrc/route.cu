@@ -1,0 +1,235 @@
+// route.cu -- per-sample top-k routing: radix select + ballot compaction.
+//
+// "Where Compute Matters: Heterogeneous Attention for Efficient Video
+// Diffusion", §3.2.2 Eq. (11)-(12): tokens with high uncertainty go dense.
+// Top-k reading: exactly k tokens per sample (k = ceil(rho*N), Eq. (14));
+// equal u are taken in increasing token index; -0.0 == +0.0.
+//
+// One CTA per sample.  The sample's u is read from HBM once (coalesced
+// 16-byte loads) into shared memory as order-preserving uint32 keys; four
+// 8-bit radix passes in shared memory find the k-th largest key K* and how
+// many keys equal to K* are taken; a last pass compacts both index lists in
+// increasing order with warp ballots and writes them as contiguous runs.
+#include "heta_internal.cuh"
+
+namespace heta {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+
+// Monotone map float -> uint32: a > b (as reals) <=> key(a) > key(b).
+// -0.0 is folded onto +0.0 first so the two compare equal.
+__device__ __forceinline__ uint32_t order_key(float f)
+{
+    uint32_t b = __float_as_uint(f);
+    if ((b & 0x7fffffffu) == 0u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t key)
+{
+    uint32_t b = (key & 0x80000000u) ? (key & 0x7fffffffu) : ~key;
+    return __uint_as_float(b);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+route_kernel(const float *__restrict__ u, int N, int k,
+             int32_t *__restrict__ dense_idx, int32_t *__restrict__ local_idx,
+             float *__restrict__ thresh, uint8_t *__restrict__ mask,
+             int32_t *status)
+{
+    extern __shared__ uint32_t keys[];
+    __shared__ uint32_t hist[256];
+    __shared__ uint32_t s_prefix, s_take;
+    __shared__ uint32_t w_gt[kWarps], w_eq[kWarps];
+    __shared__ uint32_t w_dense_before[kWarps], w_eq_before[kWarps];
+    __shared__ int s_nan;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.x;
+    const float *ub = u + (size_t)b * N;
+    if (tid == 0) s_nan = 0;
+    __syncthreads();
+
+    // ---- 1. one coalesced read of u into shared memory as keys ----------
+    bool nan_seen = false;
+    int head = 0;  // scalar elements before the first 16-byte boundary
+    {
+        uintptr_t a = reinterpret_cast<uintptr_t>(ub);
+        head = (int)(((16u - (a & 15u)) & 15u) >> 2);
+        if (head > N) head = N;
+    }
+    if (tid < head) {
+        float f = __ldg(ub + tid);
+        nan_seen |= (f != f);
+        keys[tid] = order_key(f);
+    }
+    const int n4 = (N - head) >> 2;
+    const float4 *u4 = reinterpret_cast<const float4 *>(ub + head);
+    for (int v = tid; v < n4; v += kThreads) {
+        float4 f = __ldg(u4 + v);
+        nan_seen |= (f.x != f.x) | (f.y != f.y) | (f.z != f.z) | (f.w != f.w);
+        int i = head + 4 * v;
+        keys[i] = order_key(f.x);
+        keys[i + 1] = order_key(f.y);
+        keys[i + 2] = order_key(f.z);
+        keys[i + 3] = order_key(f.w);
+    }
+    for (int i = head + 4 * n4 + tid; i < N; i += kThreads) {
+        float f = __ldg(ub + i);
+        nan_seen |= (f != f);
+        keys[i] = order_key(f);
+    }
+    if (nan_seen) s_nan = 1;
+    __syncthreads();
+    if (tid == 0 && s_nan) raise_status(status, HETA_ERR_NONFINITE);
+
+    // ---- 2. radix select of the k-th largest key --------------------------
+    uint32_t kstar = 0xffffffffu, take = 0u;  // k == 0: nothing is dense
+    if (k > 0) {
+        uint32_t prefix = 0u, remaining = (uint32_t)k;
+        const int iters = (N + kThreads - 1) / kThreads;
+        for (int pass = 0; pass < 4; ++pass) {
+            const int shift = 24 - 8 * pass;
+            const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
+            if (tid < 256) hist[tid] = 0u;
+            __syncthreads();
+            for (int it = 0; it < iters; ++it) {
+                const int i = it * kThreads + tid;
+                uint32_t digit = 256u;  // sentinel: not counted
+                if (i < N) {
+                    uint32_t key = keys[i];
+                    if ((key & hi_mask) == prefix) digit = (key >> shift) & 255u;
+                }
+                // lanes holding the same digit add once, through their leader
+                unsigned peers = __match_any_sync(0xffffffffu, digit);
+                if (digit < 256u && lane == __ffs(peers) - 1)
+                    atomicAdd(&hist[digit], (uint32_t)__popc(peers));
+            }
+            __syncthreads();
+            if (warp == 0) {
+                // lane l holds bins 255-8l .. 248-8l (descending)
+                uint32_t c[8], sum = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    c[j] = hist[255 - 8 * lane - j];
+                    sum += c[j];
+                }
+                uint32_t incl = sum;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const uint32_t before = incl - sum;
+                if (before < remaining && remaining <= incl) {
+                    uint32_t acc = before;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        if (acc < remaining && remaining <= acc + c[j]) {
+                            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+                            s_take = remaining - acc;
+                        }
+                        acc += c[j];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            remaining = s_take;
+        }
+        kstar = prefix;
+        take = remaining;
+    }
+    if (tid == 0 && thresh)
+        thresh[b] = k > 0 ? key_value(kstar) : __uint_as_float(0x7f800000u);
+
+    // ---- 3. compaction: each warp owns one contiguous segment -------------
+    const int per_lane = (N + kThreads - 1) / kThreads;
+    const int seg = 32 * per_lane;
+    const int seg_lo = warp * seg;
+    const int seg_hi = min(N, seg_lo + seg);
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int i = seg_lo + lane; i < seg_hi; i += 32) {
+        uint32_t key = keys[i];
+        n_gt += key > kstar;
+        n_eq += key == kstar;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        n_gt += __shfl_xor_sync(0xffffffffu, n_gt, o);
+        n_eq += __shfl_xor_sync(0xffffffffu, n_eq, o);
+    }
+    if (lane == 0) {
+        w_gt[warp] = n_gt;
+        w_eq[warp] = n_eq;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t eq = w_eq[lane], gt = w_gt[lane];
+        uint32_t eq_incl = eq;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t t = __shfl_up_sync(0xffffffffu, eq_incl, o);
+            if (lane >= o) eq_incl += t;
+        }
+        uint32_t eq_before = eq_incl - eq;
+        uint32_t taken_eq = take > eq_before ? min(eq, take - eq_before) : 0u;
+        uint32_t dense_here = gt + taken_eq;
+        uint32_t d_incl = dense_here;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            uint32_t t = __shfl_up_sync(0xffffffffu, d_incl, o);
+            if (lane >= o) d_incl += t;
+        }
+        w_dense_before[lane] = d_incl - dense_here;
+        w_eq_before[lane] = eq_before;
+    }
+    __syncthreads();
+
+    const unsigned lt = (1u << lane) - 1u;
+    uint32_t rd = w_dense_before[warp], re = w_eq_before[warp];
+    int32_t *dout = dense_idx + (size_t)b * k;
+    int32_t *lout = local_idx + (size_t)b * (N - k);
+    uint8_t *mout = mask ? mask + (size_t)b * N : nullptr;
+    for (int base = seg_lo; base < seg_hi; base += 32) {
+        const int i = base + lane;
+        const bool valid = i < seg_hi;
+        const uint32_t key = valid ? keys[i] : 0u;
+        const bool gt = valid && key > kstar;
+        const bool eq = valid && key == kstar;
+        const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
+        const uint32_t eq_rank = re + __popc(eq_mask & lt);
+        const bool dense = gt || (eq && eq_rank < take);
+        const unsigned d_mask = __ballot_sync(0xffffffffu, dense);
+        const uint32_t pos = rd + __popc(d_mask & lt);  // dense tokens before i
+        // the select makes |dense| == k exactly; the bounds only guard memory
+        if (dense) {
+            if (pos < (uint32_t)k) dout[pos] = i;
+        } else if (valid && (uint32_t)i - pos < (uint32_t)(N - k)) {
+            lout[i - pos] = i;
+        }
+        if (mout && valid) mout[i] = dense ? 0 : 1;
+        rd += __popc(d_mask);
+        re += __popc(eq_mask);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const float *u, int B, int N, int k, int32_t *dense_idx,
+                         int32_t *local_idx, float *thresh, uint8_t *mask,
+                         int32_t *status, cudaStream_t s)
+{
+    const size_t smem = sizeof(uint32_t) * (size_t)N;
+    cudaError_t e = cudaFuncSetAttribute(route_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(uint32_t) * kRouteMaxN));
+    if (e != cudaSuccess) return e;
+    route_kernel<<<B, kThreads, smem, s>>>(u, N, k, dense_idx, local_idx, thresh,
+                                           mask, status);
+    return cudaGetLastError();
+}
+
+}  // namespace heta

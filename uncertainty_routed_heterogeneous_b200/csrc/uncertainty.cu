@@ -1,0 +1,109 @@
+// uncertainty.cu -- the per-token uncertainty head, u = softplus(X.w + b).
+//
+// "Where Compute Matters: Heterogeneous Attention for Efficient Video
+// Diffusion", §3.2.1 Eq. (7): a lightweight branch predicts u_i >= 0 per
+// token; its output routes the next denoising step (§3.2.2, §4 Training
+// Setting).  Read here as one linear map C -> 1 followed by softplus.
+//
+// HBM-bound GEMV: every byte of X is read once with 16-byte streaming loads
+// (no L1 allocation); one warp per token row, fp32 accumulation, warp-shuffle
+// reduction, softplus in the epilogue.  w (fp32) is staged in shared memory.
+#include <cuda_bf16.h>
+
+#include "heta_internal.cuh"
+
+namespace heta {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float dot8(uint4 x, const float *w)
+{
+    const float4 w0 = *reinterpret_cast<const float4 *>(w);
+    const float4 w1 = *reinterpret_cast<const float4 *>(w + 4);
+    // a bf16 is the high half of the fp32 with the same value
+    float s = __uint_as_float(x.x << 16) * w0.x;
+    s = fmaf(__uint_as_float(x.x & 0xffff0000u), w0.y, s);
+    s = fmaf(__uint_as_float(x.y << 16), w0.z, s);
+    s = fmaf(__uint_as_float(x.y & 0xffff0000u), w0.w, s);
+    s = fmaf(__uint_as_float(x.z << 16), w1.x, s);
+    s = fmaf(__uint_as_float(x.z & 0xffff0000u), w1.y, s);
+    s = fmaf(__uint_as_float(x.w << 16), w1.z, s);
+    s = fmaf(__uint_as_float(x.w & 0xffff0000u), w1.w, s);
+    return s;
+}
+
+__device__ __forceinline__ float softplus(float z)
+{
+    return z > 0.f ? z + log1pf(expf(-z)) : log1pf(expf(z));
+}
+
+// UNROLL row-chunks of 8 elements are loaded before any is consumed, so each
+// lane keeps UNROLL 16-byte loads in flight.
+template <int UNROLL>
+__global__ void __launch_bounds__(kThreads)
+uncertainty_kernel(const uint16_t *__restrict__ X, const float *__restrict__ w,
+                   float bias, int64_t rows, int C, float *__restrict__ u)
+{
+    extern __shared__ float ws[];
+    for (int c = threadIdx.x; c < C; c += kThreads) ws[c] = w[c];
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int chunks = C >> 3;  // 8 bf16 per 16-byte chunk
+    const int64_t nwarps = (int64_t)gridDim.x * kWarps;
+    for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < rows;
+         row += nwarps) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(X + row * C);
+        float acc = 0.f;
+        for (int c0 = 0; c0 < chunks; c0 += 32 * UNROLL) {
+            uint4 v[UNROLL];
+#pragma unroll
+            for (int j = 0; j < UNROLL; ++j) {
+                const int c = c0 + j * 32 + lane;
+                v[j] = c < chunks ? ld_stream(xr + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < UNROLL; ++j) {
+                const int c = c0 + j * 32 + lane;
+                if (c < chunks) acc += dot8(v[j], ws + 8 * c);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) u[row] = softplus(acc + bias);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_uncertainty(const uint16_t *X, const float *w, float bias,
+                               int B, int N, int C, float *u, cudaStream_t s)
+{
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t rows = (int64_t)B * N;
+    const size_t smem = sizeof(float) * (size_t)C;
+    cudaError_t e = cudaFuncSetAttribute(uncertainty_kernel<6>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    // 4 CTAs of 16 warps per SM; each warp walks rows with a grid stride
+    int64_t blocks = (rows + kWarps - 1) / kWarps;
+    if (blocks > 4LL * sms) blocks = 4LL * sms;
+    uncertainty_kernel<6><<<(unsigned)blocks, kThreads, smem, s>>>(X, w, bias, rows, C, u);
+    return cudaGetLastError();
+}
+
+}  // namespace heta
