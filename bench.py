@@ -261,6 +261,8 @@ def run_heta(args, info):
     dense = torch.empty((w.B, kk), dtype=torch.int32, device=dev)
     local = torch.empty((w.B, w.N - kk), dtype=torch.int32, device=dev)
     out = torch.empty_like(d_Q)
+    ws = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, kk),
+                     dtype=torch.uint8, device=dev)
     u_next = torch.empty((w.B, w.N), dtype=torch.float32, device=dev)
     h_out = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
     h_unext = torch.empty(u_next.shape, dtype=torch.float32).pin_memory()
@@ -272,14 +274,15 @@ def run_heta(args, info):
         heta.route(d_u, kk, out=(dense, local, None, None))
         if ev is not None:
             ev[1].record()
-        heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense, out=out)
+        heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense, out=out, workspace=ws)
         if ev is not None:
             ev[2].record()
         heta.uncertainty(d_X, d_w, 0.0, out=u_next)
         if ev is not None:
             ev[3].record()
 
-    launches_per_step = 1 + (1 if kk > 0 else 0) + (1 if kk < w.N else 0) + 1
+    # route, the persistent attention kernel, the head (plus one workspace memset)
+    launches_per_step = 3
     flops = heta.attention_flops(w.B, w.H, w.d, w.N, kk, w.M)
 
     sampler = ClockSampler(info.local_rank)
@@ -311,13 +314,15 @@ def run_heta(args, info):
     dense_cmp = None
     if not args.no_dense_compare:
         all_idx = torch.arange(w.N, dtype=torch.int32, device=dev).repeat(w.B, 1).contiguous()
-        heta.attention(d_Q, d_K, d_V, w.grid, w.win, all_idx, out=out)
+        ws_full = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, w.N),
+                              dtype=torch.uint8, device=dev)
+        heta.attention(d_Q, d_K, d_V, w.grid, w.win, all_idx, out=out, workspace=ws_full)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         reps = 3
         e0.record()
         for _ in range(reps):
-            heta.attention(d_Q, d_K, d_V, w.grid, w.win, all_idx, out=out)
+            heta.attention(d_Q, d_K, d_V, w.grid, w.win, all_idx, out=out, workspace=ws_full)
         e1.record()
         torch.cuda.synchronize()
         full_ms = e0.elapsed_time(e1) / reps
@@ -373,7 +378,7 @@ def run_heta(args, info):
         "config": config_of(base, info.world),
         "attention_tflops": tflops,
         "kernel_ms": {"route": route_ms, "attention": attn_ms, "head": head_ms},
-        "roofline": {"bound": "tensor", "kernel": "heta_attention (dense + local kernels)",
+        "roofline": {"bound": "tensor", "kernel": "attn_tc_kernel (persistent; dense + local items)",
                      "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "frac_of_burst": tflops / peaks["bf16_tflops"],
                      "peak_source": "%s sustained bf16 (cuBLAS)" % peaks["source"],

@@ -96,6 +96,21 @@ HETA_API heta_status heta_route(const float *u, int B, int N, int k,
                        int32_t *status_dev, void *stream);
 
 /*
+ * heta_attention_workspace_size -- device scratch one heta_attention call
+ * needs for these sizes (host-only; touches no device).
+ *
+ * The scratch holds the work-item counter of the persistent kernel and, when
+ * the dense rows' key range is split in two to keep all SMs busy, the
+ * partial results the two halves merge (fp32, about 1 KB per dense row and
+ * half for d = 64).  At the Wan2.1-1.3B shape with rho = 0.2 that is about
+ * 83 MB; when no split is needed it is 256 bytes.  Same argument rules as
+ * heta_attention; *bytes is only written on HETA_OK.
+ */
+HETA_API heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg,
+                                                   int Wg, int wt, int wh, int ww, int k,
+                                                   size_t *bytes);
+
+/*
  * heta_attention -- routed heterogeneous self-attention (Eq. (2), (3), (13)).
  *
  * For every sample b, head h and token i:
@@ -113,16 +128,25 @@ HETA_API heta_status heta_route(const float *u, int B, int N, int k,
  *              of range or out of order give unspecified rows.
  *   out        [B,H,N,d] bf16 out; every row is written exactly once.
  *   scale      softmax scale, normally 1/sqrt(d).
+ *   workspace  device scratch of at least heta_attention_workspace_size()
+ *              bytes, 16-byte aligned, owned by the caller; its contents on
+ *              entry do not matter and are garbage on return.  Calls that
+ *              may run at the same time need separate workspaces.
  *
- * Requires d in {64, 128}; odd wt, wh, ww with 1 <= w_a <= extent_a;
- * N = Tg*Hg*Wg; 0 <= k <= N; B*H*N*d < 2^40.  Other d or even windows give
- * HETA_ERR_UNSUPPORTED.
+ * One persistent kernel launch (plus a small memset of the workspace's
+ * counters) on `stream`.  Requires d in {64, 128}; odd wt, wh, ww with
+ * 1 <= w_a <= extent_a; N = Tg*Hg*Wg; 0 <= k <= N; B*H < 65536;
+ * B*H*N*d < 2^40.  Other d or even windows give HETA_ERR_UNSUPPORTED.  A
+ * wait inside the kernel that exceeds about 2 s raises status_dev to
+ * HETA_ERR_TIMEOUT and the kernel returns (the context stays usable).
  */
 HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
-                           const uint16_t *V, int B, int H, int d,
-                           int Tg, int Hg, int Wg, int wt, int wh, int ww,
-                           float scale, const int32_t *dense_idx, int k,
-                           uint16_t *out, int32_t *status_dev, void *stream);
+                                    const uint16_t *V, int B, int H, int d,
+                                    int Tg, int Hg, int Wg, int wt, int wh, int ww,
+                                    float scale, const int32_t *dense_idx, int k,
+                                    uint16_t *out, void *workspace,
+                                    size_t workspace_bytes, int32_t *status_dev,
+                                    void *stream);
 
 /*
  * heta_uncertainty -- the lightweight per-token uncertainty head (Eq. (7)).

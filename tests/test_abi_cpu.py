@@ -34,7 +34,7 @@ def declared_symbols():
 def test_header_declares_the_three_path_calls():
     names = declared_symbols()
     assert {"heta_route", "heta_attention", "heta_uncertainty", "heta_dense_count",
-            "heta_status_string", "heta_version"} <= names
+            "heta_status_string", "heta_version", "heta_attention_workspace_size"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -72,7 +72,8 @@ def test_host_validation_returns_before_any_launch(lib):
     # misaligned pointer
     odd = ctypes.c_void_p((1 << 20) + 4)
     assert lib.heta_route(odd, 1, 10, 2, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
-    args = [fake, fake, fake, 1, 2, 128, 4, 8, 8, 3, 3, 3, ctypes.c_float(0.1), fake, 3, fake, N, N]
+    args = [fake, fake, fake, 1, 2, 128, 4, 8, 8, 3, 3, 3, ctypes.c_float(0.1), fake, 3, fake,
+            fake, 1 << 30, N, N]
     bad_d = list(args)
     bad_d[5] = 96
     assert lib.heta_attention(*bad_d) == heta.HETA_ERR_UNSUPPORTED
@@ -88,6 +89,12 @@ def test_host_validation_returns_before_any_launch(lib):
     bad_scale = list(args)
     bad_scale[12] = ctypes.c_float(float("nan"))
     assert lib.heta_attention(*bad_scale) == heta.HETA_ERR_INVALID_ARG
+    small_ws = list(args)
+    small_ws[17] = 16
+    assert lib.heta_attention(*small_ws) == heta.HETA_ERR_INVALID_ARG
+    no_ws = list(args)
+    no_ws[16] = N
+    assert lib.heta_attention(*no_ws) == heta.HETA_ERR_INVALID_ARG
     assert lib.heta_uncertainty(fake, fake, ctypes.c_float(0.0), 1, 10, 12, fake, N, N) == \
         heta.HETA_ERR_INVALID_ARG
     assert lib.heta_uncertainty(fake, fake, ctypes.c_float(0.0), 1, 10, 32768, fake, N, N) == \
@@ -107,3 +114,18 @@ def test_flop_model_matches_the_papers_reduction():
     het = heta.attention_flops(1, 12, 128, N, k, M)
     assert abs(full / het - 4.87) < 0.02
     assert het == 4 * 128 * 12 * (k * N + (N - k) * M)
+
+
+def test_workspace_size(lib):
+    """Counter-only scratch when the dense pairs fill the SMs; a split merge buffer
+    when they do not (Wan2.1 shape at rho = 0.2)."""
+    full = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), 32760)
+    assert full == 256
+    k = heta.dense_count(32760, 0.2)
+    part = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k)
+    pairs = 12 * (((k + 127) // 128 + 1) // 2)
+    assert part >= pairs * 2 * 2 * 128 * (128 * 4 + 8)
+    assert part < 100 * 2 ** 20
+    assert heta.attention_workspace_size(1, 2, 64, (4, 8, 8), (3, 3, 3), 0) == 256
+    with pytest.raises(heta.HetaError):
+        heta.attention_workspace_size(1, 2, 96, (4, 8, 8), (3, 3, 3), 10)

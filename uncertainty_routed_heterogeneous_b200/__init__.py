@@ -18,6 +18,7 @@ import math
 import os
 
 __all__ = ["load", "HetaError", "dense_count", "route", "attention", "uncertainty",
+           "attention_workspace_size",
            "status_string", "attention_flops", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libheta.so")
@@ -58,7 +59,10 @@ def load():
     lib.heta_dense_count.restype = i
     lib.heta_route.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, vp]
     lib.heta_route.restype = i
-    lib.heta_attention.argtypes = [vp, vp, vp] + [i] * 9 + [f, vp, i, vp, vp, vp]
+    lib.heta_attention_workspace_size.argtypes = [i] * 10 + [ctypes.POINTER(ctypes.c_size_t)]
+    lib.heta_attention_workspace_size.restype = i
+    lib.heta_attention.argtypes = [vp, vp, vp] + [i] * 9 + [f, vp, i, vp, vp, ctypes.c_size_t,
+                                                            vp, vp]
     lib.heta_attention.restype = i
     lib.heta_uncertainty.argtypes = [vp, vp, f, i, i, i, vp, vp, vp]
     lib.heta_uncertainty.restype = i
@@ -131,12 +135,24 @@ def route(u, k: int, *, out=None, want_thresh=False, want_mask=False, status=Non
     return dense, local, thresh, mask
 
 
-def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=None):
+def attention_workspace_size(B, H, d, grid, win, k) -> int:
+    """Bytes of device scratch one ``attention`` call needs for these sizes."""
+    n = ctypes.c_size_t(0)
+    _check(load().heta_attention_workspace_size(int(B), int(H), int(d), grid[0], grid[1],
+                                                grid[2], win[0], win[1], win[2], int(k),
+                                                ctypes.byref(n)),
+           "heta_attention_workspace_size")
+    return int(n.value)
+
+
+def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=None,
+              workspace=None):
     """Routed heterogeneous attention (``heta_attention``).
 
     Q, K, V: [B,H,N,d] bfloat16 CUDA; grid = (Tg, Hg, Wg) with N = Tg*Hg*Wg;
     win = (wt, wh, ww) odd; dense_idx: [B,k] int32 CUDA, increasing.
-    Returns out [B,H,N,d] bfloat16.
+    ``workspace``: a uint8 CUDA tensor of at least ``attention_workspace_size``
+    bytes (allocated here when omitted).  Returns out [B,H,N,d] bfloat16.
     """
     import torch
     pq = _dev(Q, torch.bfloat16, "Q", 4)
@@ -157,9 +173,13 @@ def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=Non
     po = _dev(out, torch.bfloat16, "out", 4)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    need = attention_workspace_size(B, H, d, grid, win, k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=Q.device)
+    pw = _dev(workspace, torch.uint8, "workspace", 1)
     rc = load().heta_attention(pq, pk, pv, B, H, d, Tg, Hg, Wg, win[0], win[1], win[2],
-                               float(scale), pd if k > 0 else None, k, po, _opt(status),
-                               _stream())
+                               float(scale), pd if k > 0 else None, k, po, pw,
+                               workspace.numel(), _opt(status), _stream())
     _check(rc, "heta_attention")
     return out
 

@@ -5,23 +5,28 @@
 // rows, Eq. (3) attention over a clamped 3D (t,h,w) window for every other
 // row, merged row by row as in Eq. (13); Eq. (14) is the cost model.
 //
-// One kernel template, two modes:
-//   DENSE: a CTA owns two 128-row query tiles gathered through dense_idx and
-//          streams all N keys of its (b,h) in 128-key K/V tiles.
-//   LOCAL: a CTA owns two 2x8x8 query boxes of the latent grid; each box
-//          streams the K/V sub-tiles (1x8x16 keys each) that cover the union
-//          of its rows' windows, with a per-element window mask.  Rows whose
-//          token is dense are computed but not stored.
-// Both modes: K/V tiles arrive by TMA (128-byte swizzle) into a shared-memory
-// ring; one thread issues tcgen05.mma with fp32 accumulators in TMEM
-// (S = Q K^T per tile, O += P V with P read back from TMEM); two softmax
-// warpgroups (one thread per query row) ping-pong on the two tiles with an
-// online softmax in the log2 domain.  The O rescale is skipped unless the
-// running row maximum grows by more than 2^8.  Epilogue: O / l in bf16,
-// stored straight to the row's place in out (the Eq. (13) scatter).
+// One persistent kernel runs both kinds of work item, handed out in order by
+// an atomic counter (dense items first: they are the long ones):
+//   DENSE item: two 128-row query tiles of one (b,h), gathered through
+//               dense_idx, against one contiguous range of 128-key K/V tiles
+//               (all N keys, or half of them when the host splits the key
+//               range to balance the SMs; the second half to finish merges
+//               the other's partial result -- no CTA ever waits on another).
+//   LOCAL item: two 2x8x8 query boxes of the latent grid; each box streams
+//               the 1x8x16-key K/V sub-tiles that cover its rows' windows,
+//               with a per-element window mask.  Rows whose token is dense
+//               are computed but not stored.
+// Per CTA (one per SM): a TMA producer warp fills a shared-memory ring of K/V
+// tiles (128-byte swizzle) and loads LOCAL query boxes; one thread issues
+// tcgen05.mma with fp32 accumulators in TMEM (S = Q K^T, O += P V with P read
+// back from TMEM); two softmax warpgroups (one thread per query row) ping-pong
+// on the two tiles with an online softmax in the log2 domain, rescaling O
+// only when a row maximum grows by more than 2^8; a flags warp finds the
+// dense tokens inside LOCAL boxes.  Epilogue: O / l in bf16, stored straight
+// to the row's place in out (the Eq. (13) scatter).
 //
-// Every mbarrier wait is bounded; on expiry the kernel raises
-// HETA_ERR_TIMEOUT in status, unwinds, drains its copies and frees TMEM.
+// Every wait is bounded; on expiry the kernel raises HETA_ERR_TIMEOUT in
+// status, unwinds, drains its copies and MMAs and frees TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -36,12 +41,13 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 384;          // 12 warps
-constexpr int kTileRows = 128;         // query rows per tile (MMA M)
-constexpr int kTileKeys = 128;         // keys per K/V tile (MMA N of S)
-constexpr int kRingBytes = 128 * 1024; // K/V ring
+constexpr int kThreads = 384;           // 12 warps
+constexpr int kTileRows = 128;          // query rows per tile (MMA M)
+constexpr int kTileKeys = 128;          // keys per K/V tile (MMA N of S)
+constexpr int kRingBytes = 128 * 1024;  // K/V ring
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr float kRescaleLog2 = 8.0f;   // rescale O only when the max grows > 2^8
+constexpr float kRescaleLog2 = 8.0f;    // rescale O only when the max grows > 2^8
+constexpr int kQueue = 4;               // work-item queue depth
 
 // query box (LOCAL) and key sub-tile
 constexpr int kBoxT = 2, kBoxH = 8, kBoxW = 8;
@@ -51,6 +57,8 @@ enum { DENSE = 0, LOCAL = 1 };
 
 // warp roles
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpFlags = 2, kWarpSoftmax0 = 4;
+// consumers of the item queue: MMA thread, 256 softmax threads, flags warp
+constexpr uint32_t kItemConsumers = 1 + 256 + 32;
 
 struct Params {
     const uint16_t *Q;
@@ -60,16 +68,22 @@ struct Params {
     int B, H, N, k;
     int Tg, Hg, Wg, wt, wh, ww;
     float scale_log2;
-    int tiles;   // DENSE: query tiles per (b,h); LOCAL: boxes per (b,h)
-    int n_kv;    // K/V tiles each query tile streams
-    int nbh, nbw;            // LOCAL: boxes along h and w
-    int nkt, nkh, nkw;       // LOCAL: K/V sub-tiles along t, h, w
+    // DENSE items
+    int tiles_d, pairs_d, nsplit, n_kv_d, kv_per_split, n_dense_items;
+    // LOCAL items
+    int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
+    int total_items;
+    // scratch
+    int *counter;     // next work item
+    int *fix_count;   // [B*H*pairs_d][2] split arrivals
+    float *part_o;    // [B*H*pairs_d][nsplit][2][128][D]
+    float2 *part_ml;  // [B*H*pairs_d][nsplit][2][128] (m, l)
 };
 
 template <int D>
 struct Cfg {
-    static constexpr int kSub = D / 64;                     // 128-byte column blocks
-    static constexpr int kTileBytes = kTileRows * D * 2;    // one Q/K/V tile
+    static constexpr int kSub = D / 64;                   // 128-byte column blocks
+    static constexpr int kTileBytes = kTileRows * D * 2;  // one Q/K/V tile
     static constexpr int kStages = kRingBytes / kTileBytes;
     static constexpr int kQBytes = 2 * kTileBytes;
     static constexpr int kSmem = kQBytes + kRingBytes + 1024;  // + alignment slack
@@ -95,17 +109,64 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+__device__ __forceinline__ void named_bar(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// One work item, decoded from its index.
+struct Item {
+    int mode;        // DENSE or LOCAL
+    int bh;          // b*H + h
+    int b;
+    int tile[2];     // query tile (DENSE) / box (LOCAL) of each slot
+    int kv_lo, n;    // K/V tiles [kv_lo, kv_lo + n)
+    int split;       // DENSE: which key range
+    int pair_id;     // DENSE: global pair index (for the split merge)
+};
+
+__device__ __forceinline__ Item decode(const Params &p, int id)
+{
+    Item it;
+    if (id < p.n_dense_items) {
+        const int per_bh = p.pairs_d * p.nsplit;
+        it.mode = DENSE;
+        it.bh = id / per_bh;
+        const int r = id % per_bh;
+        const int pair = r / p.nsplit;
+        it.split = r % p.nsplit;
+        it.pair_id = it.bh * p.pairs_d + pair;
+        it.tile[0] = 2 * pair;
+        it.tile[1] = 2 * pair + 1;
+        it.kv_lo = it.split * p.kv_per_split;
+        it.n = min(p.n_kv_d, it.kv_lo + p.kv_per_split) - it.kv_lo;
+    } else {
+        const int id2 = id - p.n_dense_items;
+        it.mode = LOCAL;
+        it.bh = id2 / p.pairs_l;
+        const int pair = id2 % p.pairs_l;
+        it.split = 0;
+        it.pair_id = 0;
+        it.tile[0] = 2 * pair;
+        it.tile[1] = 2 * pair + 1;
+        it.kv_lo = 0;
+        it.n = p.n_kv_l;
+    }
+    it.b = it.bh / p.H;
+    return it;
+}
+
 // Geometry of one LOCAL query box and the origin of its K/V cover.
 struct Box {
-    int t0, h0, w0;       // box origin
-    int tlo, hlo, wlo;    // origin of the K/V cover
+    int t0, h0, w0;     // box origin
+    int tlo, hlo, wlo;  // origin of the K/V cover
     bool active;
 };
 
 __device__ __forceinline__ Box local_box(const Params &p, int box)
 {
     Box x;
-    x.active = box < p.tiles;
+    x.active = box < p.tiles_l;
     const int bb = x.active ? box : 0;
     const int bw = bb % p.nbw, bh = (bb / p.nbw) % p.nbh, bt = bb / (p.nbw * p.nbh);
     x.t0 = bt * kBoxT;
@@ -119,16 +180,21 @@ __device__ __forceinline__ Box local_box(const Params &p, int box)
 
 struct Shared {
     uint64_t kv_full[16], kv_empty[16];
-    uint64_t q_full[2], s_full[2], p_full[2], o_done[2], flags_ready, drain;
+    uint64_t item_full[kQueue], item_empty[kQueue];
+    uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_done[2], o_empty[2];
+    uint64_t flags_full, flags_empty, drain;
+    int item_q[kQueue];
     uint32_t tmem_base;
     int abort;
+    int fix_old[2];
     uint8_t no_store[2][kTileRows];  // LOCAL: row holds a dense token
 };
 
-template <int D, int MODE>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-               const Params p)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__ CUtensorMap tmV3,
+               const __grid_constant__ CUtensorMap tmK5, const __grid_constant__ CUtensorMap tmV5,
+               const __grid_constant__ CUtensorMap tmQ5, const Params p)
 {
     using C = Cfg<D>;
     extern __shared__ __align__(1024) uint8_t dyn_smem[];
@@ -136,26 +202,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
 
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-    uint8_t *q_smem = smem;                      // [2][kSub][128 rows][128 B]
-    uint8_t *ring = smem + C::kQBytes;           // [kStages][kSub][128 rows][128 B]
+    uint8_t *q_smem = smem;             // [2][kSub][128 rows][128 B]
+    uint8_t *ring = smem + C::kQBytes;  // [kStages][kSub][128 rows][128 B]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int pair = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int64_t bh = (int64_t)b * p.H + h;
-    const int n = p.n_kv;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(smem_addr(&sh.kv_full[s]), 1);
             mbar_init(smem_addr(&sh.kv_empty[s]), 1);
         }
+        for (int q = 0; q < kQueue; ++q) {
+            mbar_init(smem_addr(&sh.item_full[q]), 1);
+            mbar_init(smem_addr(&sh.item_empty[q]), kItemConsumers);
+        }
         for (int t = 0; t < 2; ++t) {
-            mbar_init(smem_addr(&sh.q_full[t]), kTileRows);
+            mbar_init(smem_addr(&sh.q_full[t]), 1);
+            mbar_init(smem_addr(&sh.q_empty[t]), 1);
             mbar_init(smem_addr(&sh.s_full[t]), 1);
             mbar_init(smem_addr(&sh.p_full[t]), kTileRows);
             mbar_init(smem_addr(&sh.o_done[t]), 1);
+            mbar_init(smem_addr(&sh.o_empty[t]), kTileRows);
         }
-        mbar_init(smem_addr(&sh.flags_ready), 1);
+        mbar_init(smem_addr(&sh.flags_full), 1);
+        mbar_init(smem_addr(&sh.flags_empty), 2 * kTileRows);
         mbar_init(smem_addr(&sh.drain), 1);
         sh.abort = 0;
         fence_mbar_init();
@@ -174,97 +244,135 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
     auto fail = [&]() {
         if (atomicExch(&sh.abort, 1) == 0) raise_status(p.status, HETA_ERR_TIMEOUT);
     };
-
-    // the two query tiles of this CTA
-    const int tile0 = 2 * pair, tile1 = 2 * pair + 1;
+    auto wait = [&](uint64_t &bar, uint32_t parity) -> bool {
+        return mbar_wait(smem_addr(&bar), parity, abort, kWaitLimitNs);
+    };
+    // reads queue entry qi (blocking); every consumer arrives on item_empty
+    auto pop_item = [&](uint32_t qi, bool &ok) -> int {
+        const int slot = qi % kQueue;
+        if (!wait(sh.item_full[slot], (qi / kQueue) & 1u)) {
+            ok = false;
+            return -1;
+        }
+        const int id = *reinterpret_cast<volatile int *>(&sh.item_q[slot]);
+        mbar_arrive(smem_addr(&sh.item_empty[slot]));
+        return id;
+    };
 
     if (warp == kWarpTma) {
-        // ------------------------------------------------------------ producer
+        // ============================================================ producer
         if (lane == 0) {
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            Box bx[2];
-            if (MODE == LOCAL) {
-                bx[0] = local_box(p, tile0);
-                bx[1] = local_box(p, tile1);
-            }
-            int issued = 0;
+            prefetch_tmap(&tmK3);
+            prefetch_tmap(&tmV3);
+            prefetch_tmap(&tmK5);
+            prefetch_tmap(&tmV5);
+            prefetch_tmap(&tmQ5);
+            uint32_t issued = 0, qi = 0, items = 0;
             bool ok = true;
-            // one element of the tile sequence the MMA thread consumes in order
-            auto load = [&](bool is_v, int slot, int j) {
-                if (!ok) return;
-                const int s = issued;
-                const int stage = s % C::kStages;
-                const uint32_t use = (uint32_t)(s / C::kStages);
-                if (!mbar_wait(smem_addr(&sh.kv_empty[stage]), (use & 1u) ^ 1u, abort,
-                               kWaitLimitNs)) {
-                    ok = false;
-                    return;
+            int id = atomicAdd(p.counter, 1);
+            while (ok) {
+                if (id >= p.total_items) id = -1;
+                const int next = id >= 0 ? atomicAdd(p.counter, 1) : -1;
+                // publish the item
+                {
+                    const int slot = qi % kQueue;
+                    if (!wait(sh.item_empty[slot], ((qi / kQueue) & 1u) ^ 1u)) { ok = false; break; }
+                    sh.item_q[slot] = id;
+                    mbar_arrive(smem_addr(&sh.item_full[slot]));
+                    ++qi;
                 }
-                const uint32_t full = smem_addr(&sh.kv_full[stage]);
-                mbar_arrive_expect_tx(full, C::kTileBytes);
-                const uint32_t dst = smem_addr(ring + (size_t)stage * C::kTileBytes);
-                const CUtensorMap *m = is_v ? &tmV : &tmK;
-                for (int c = 0; c < C::kSub; ++c) {
-                    if (MODE == DENSE) {
-                        tma_load_3d(dst + c * 16384, m, full, 64 * c, j * kTileKeys, (int)bh);
-                    } else {
-                        const Box &x = bx[slot];
-                        const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh,
-                                  jw = j % p.nkw;
-                        tma_load_5d(dst + c * 16384, m, full, 64 * c, x.wlo + jw * kKvW,
-                                    x.hlo + jh * kKvH, x.tlo + jt, (int)bh);
+                if (id < 0) break;
+                const Item it = decode(p, id);
+                Box bx[2];
+                if (it.mode == LOCAL) {
+                    bx[0] = local_box(p, it.tile[0]);
+                    bx[1] = local_box(p, it.tile[1]);
+                }
+                // the query buffers are free once the last S of the previous item is done
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (items > 0 && !wait(sh.q_empty[t], (items - 1) & 1u)) ok = false;
+                    if (ok && it.mode == LOCAL) {
+                        const uint32_t full = smem_addr(&sh.q_full[t]);
+                        mbar_arrive_expect_tx(full, C::kTileBytes);
+                        const uint32_t dst = smem_addr(q_smem + t * C::kTileBytes);
+                        for (int c = 0; c < C::kSub; ++c)
+                            tma_load_5d(dst + c * 16384, &tmQ5, full, 64 * c, bx[t].w0,
+                                        bx[t].h0, bx[t].t0, it.bh);
                     }
                 }
-                ++issued;
-            };
-            if (MODE == DENSE) {
-                // K0, then per j: V_j, K_{j+1}
-                load(false, 0, 0);
-                for (int j = 0; j < n; ++j) {
-                    load(true, 0, j);
-                    if (j + 1 < n) load(false, 0, j + 1);
+                // one element of the K/V tile sequence the MMA thread consumes in order
+                auto load = [&](bool is_v, int slot, int j) {
+                    if (!ok) return;
+                    const uint32_t s = issued;
+                    const int stage = s % C::kStages;
+                    if (!wait(sh.kv_empty[stage], ((s / C::kStages) & 1u) ^ 1u)) {
+                        ok = false;
+                        return;
+                    }
+                    const uint32_t full = smem_addr(&sh.kv_full[stage]);
+                    mbar_arrive_expect_tx(full, C::kTileBytes);
+                    const uint32_t dst = smem_addr(ring + (size_t)stage * C::kTileBytes);
+                    for (int c = 0; c < C::kSub; ++c) {
+                        if (it.mode == DENSE) {
+                            tma_load_3d(dst + c * 16384, is_v ? &tmV3 : &tmK3, full, 64 * c,
+                                        (it.kv_lo + j) * kTileKeys, it.bh);
+                        } else {
+                            const Box &x = bx[slot];
+                            const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh,
+                                      jw = j % p.nkw;
+                            tma_load_5d(dst + c * 16384, is_v ? &tmV5 : &tmK5, full, 64 * c,
+                                        x.wlo + jw * kKvW, x.hlo + jh * kKvH, x.tlo + jt, it.bh);
+                        }
+                    }
+                    ++issued;
+                };
+                const int n = it.n;
+                if (it.mode == DENSE) {
+                    // K0, then per j: V_j, K_{j+1}   (both query tiles share them)
+                    load(false, 0, 0);
+                    for (int j = 0; j < n; ++j) {
+                        load(true, 0, j);
+                        if (j + 1 < n) load(false, 0, j + 1);
+                    }
+                } else {
+                    // K0_0, K1_0, then per j: V0_j, K0_{j+1}, V1_j, K1_{j+1}
+                    load(false, 0, 0);
+                    load(false, 1, 0);
+                    for (int j = 0; j < n; ++j) {
+                        load(true, 0, j);
+                        if (j + 1 < n) load(false, 0, j + 1);
+                        load(true, 1, j);
+                        if (j + 1 < n) load(false, 1, j + 1);
+                    }
                 }
-            } else {
-                // K0_0, K1_0, then per j: V0_j, K0_{j+1}, V1_j, K1_{j+1}
-                load(false, 0, 0);
-                load(false, 1, 0);
-                for (int j = 0; j < n; ++j) {
-                    load(true, 0, j);
-                    if (j + 1 < n) load(false, 0, j + 1);
-                    load(true, 1, j);
-                    if (j + 1 < n) load(false, 1, j + 1);
-                }
+                ++items;
+                id = next;
             }
             if (!ok) fail();
             // drain: every issued copy has landed before the CTA may exit
-            for (int s = max(0, issued - C::kStages); s < issued; ++s) {
-                const int stage = s % C::kStages;
-                const uint32_t use = (uint32_t)(s / C::kStages);
-                mbar_wait(smem_addr(&sh.kv_full[stage]), use & 1u, abort, kWaitLimitNs);
-            }
+            for (uint32_t s = issued > (uint32_t)C::kStages ? issued - C::kStages : 0; s < issued; ++s)
+                wait(sh.kv_full[s % C::kStages], (s / C::kStages) & 1u);
         }
     } else if (warp == kWarpMma) {
-        // ------------------------------------------------------------ MMA issuer
+        // ============================================================ MMA issuer
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, kTileKeys, false);
             const uint32_t id_o = idesc_bf16(128, D, true);
             const uint32_t q_addr[2] = {smem_addr(q_smem), smem_addr(q_smem + C::kTileBytes)};
             const uint32_t colS[2] = {C::kColS0, C::kColS1};
             const uint32_t colO[2] = {C::kColO0, C::kColO1};
-            int s = 0;  // ring sequence position
+            uint32_t s = 0, qi = 0, items = 0;
             bool ok = true;
-            auto wait_full = [&](int seq) -> uint32_t {
+            auto wait_full = [&](uint32_t seq) -> uint32_t {
                 const int stage = seq % C::kStages;
-                if (!mbar_wait(smem_addr(&sh.kv_full[stage]), (uint32_t)(seq / C::kStages) & 1u,
-                               abort, kWaitLimitNs)) {
+                if (!wait(sh.kv_full[stage], (seq / C::kStages) & 1u)) {
                     ok = false;
                     return 0;
                 }
                 tc_fence_after();
                 return smem_addr(ring + (size_t)stage * C::kTileBytes);
             };
-            auto release = [&](int seq) { mma_commit(smem_addr(&sh.kv_empty[seq % C::kStages])); };
+            auto release = [&](uint32_t seq) { mma_commit(smem_addr(&sh.kv_empty[seq % C::kStages])); };
             // S_t = Q_t K^T : M=128, N=128 keys, K=D (both operands K-major)
             auto issue_s = [&](int t, uint32_t k_addr) {
 #pragma unroll
@@ -283,94 +391,99 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                            (first && kk == 0) ? 0u : 1u);
                 }
             };
-            for (int t = 0; t < 2 && ok; ++t) {
-                if (!mbar_wait(smem_addr(&sh.q_full[t]), 0, abort, kWaitLimitNs)) ok = false;
-            }
-            tc_fence_after();
-            if (ok) {
-                if (MODE == DENSE) {
+            uint32_t pc[2] = {0, 0};  // p_full phases consumed per slot
+            while (ok) {
+                const int id = pop_item(qi++, ok);
+                if (!ok || id < 0) break;
+                const Item it = decode(p, id);
+                const int n = it.n;
+                const bool dense = it.mode == DENSE;
+                for (int t = 0; t < 2 && ok; ++t)
+                    if (!wait(sh.q_full[t], items & 1u)) ok = false;
+                if (!ok) break;
+                tc_fence_after();
+                // first S of each slot
+                if (dense) {
                     const uint32_t k0 = wait_full(s);
-                    if (ok) {
-                        issue_s(0, k0);
-                        mma_commit(smem_addr(&sh.s_full[0]));
-                        issue_s(1, k0);
-                        mma_commit(smem_addr(&sh.s_full[1]));
-                        release(s);
-                        ++s;
-                    }
+                    if (!ok) break;
+                    issue_s(0, k0);
+                    mma_commit(smem_addr(&sh.s_full[0]));
+                    issue_s(1, k0);
+                    mma_commit(smem_addr(&sh.s_full[1]));
+                    release(s++);
                 } else {
                     for (int t = 0; t < 2 && ok; ++t) {
                         const uint32_t kt = wait_full(s);
                         if (!ok) break;
                         issue_s(t, kt);
                         mma_commit(smem_addr(&sh.s_full[t]));
-                        release(s);
-                        ++s;
+                        release(s++);
                     }
+                    if (!ok) break;
                 }
-            }
-            for (int j = 0; j < n && ok; ++j) {
-                const bool last = j + 1 == n;
-                uint32_t v_addr = 0, kn_addr = 0;
-                int v_seq = 0, kn_seq = 0;
-                for (int t = 0; t < 2 && ok; ++t) {
-                    // V tile for this slot
-                    if (MODE == DENSE) {
-                        if (t == 0) {
+                if (n == 1) {
+                    mma_commit(smem_addr(&sh.q_empty[0]));
+                    mma_commit(smem_addr(&sh.q_empty[1]));
+                }
+                for (int j = 0; j < n && ok; ++j) {
+                    const bool last = j + 1 == n;
+                    uint32_t v_addr = 0, kn_addr = 0, v_seq = 0, kn_seq = 0;
+                    for (int t = 0; t < 2 && ok; ++t) {
+                        if (!dense || t == 0) {
                             v_seq = s++;
                             v_addr = wait_full(v_seq);
                             if (!ok) break;
                         }
-                    } else {
-                        v_seq = s++;
-                        v_addr = wait_full(v_seq);
-                        if (!ok) break;
-                    }
-                    if (!mbar_wait(smem_addr(&sh.p_full[t]), (uint32_t)j & 1u, abort,
-                                   kWaitLimitNs)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_pv(t, v_addr, j == 0);
-                    if (MODE == LOCAL) release(v_seq);
-                    if (MODE == DENSE && t == 1) release(v_seq);
-                    if (last) {
-                        mma_commit(smem_addr(&sh.o_done[t]));
-                        continue;
-                    }
-                    // next S for this slot
-                    if (MODE == DENSE) {
-                        if (t == 0) {
+                        if (!wait(sh.p_full[t], pc[t] & 1u)) { ok = false; break; }
+                        ++pc[t];
+                        tc_fence_after();
+                        // the previous item's epilogue must have read O_t before it is overwritten
+                        if (j == 0 && items > 0 && !wait(sh.o_empty[t], (items - 1) & 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        issue_pv(t, v_addr, j == 0);
+                        if (!dense || t == 1) release(v_seq);
+                        if (last) {
+                            mma_commit(smem_addr(&sh.o_done[t]));
+                            continue;
+                        }
+                        if (!dense || t == 0) {
                             kn_seq = s++;
                             kn_addr = wait_full(kn_seq);
                             if (!ok) break;
                         }
-                    } else {
-                        kn_seq = s++;
-                        kn_addr = wait_full(kn_seq);
-                        if (!ok) break;
+                        issue_s(t, kn_addr);
+                        mma_commit(smem_addr(&sh.s_full[t]));
+                        if (!dense || t == 1) release(kn_seq);
+                        if (j + 2 == n) mma_commit(smem_addr(&sh.q_empty[t]));
                     }
-                    issue_s(t, kn_addr);
-                    mma_commit(smem_addr(&sh.s_full[t]));
-                    if (MODE == LOCAL || t == 1) release(kn_seq);
                 }
+                ++items;
             }
             if (!ok) fail();
             // drain every MMA this thread issued before TMEM can be freed
             mma_commit(smem_addr(&sh.drain));
-            mbar_wait(smem_addr(&sh.drain), 0, abort, kWaitLimitNs);
+            wait(sh.drain, 0);
         }
     } else if (warp == kWarpFlags) {
-        // ------------------------------------------------- LOCAL: dense rows
-        if (MODE == LOCAL) {
+        // ============================================ flags: dense rows of LOCAL boxes
+        uint32_t qi = 0, lc = 0;
+        bool ok = true;
+        while (ok) {
+            const int id = pop_item(qi++, ok);
+            if (!ok || id < 0) break;
+            const Item it = decode(p, id);
+            if (it.mode != LOCAL) continue;
+            if (!wait(sh.flags_empty, (lc & 1u) ^ 1u)) { ok = false; break; }
             for (int t = 0; t < 2; ++t)
                 for (int r = lane; r < kTileRows; r += 32) sh.no_store[t][r] = 0;
             __syncwarp();
-            const int32_t *dl = p.dense_idx + (int64_t)b * p.k;
+            const int32_t *dl = p.dense_idx + (int64_t)it.b * p.k;
             const int HW = p.Hg * p.Wg;
             for (int t = 0; t < 2 && p.k > 0; ++t) {
-                const Box x = local_box(p, t == 0 ? tile0 : tile1);
+                const Box x = local_box(p, it.tile[t]);
                 if (!x.active) continue;
                 const int lo_tok = (x.t0 * p.Hg + x.h0) * p.Wg + x.w0;
                 const int hi_tok = (min(x.t0 + kBoxT, p.Tg) - 1) * HW +
@@ -382,8 +495,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                     const int step = (hi - lo + 31) / 32;
                     const int pos = lo + lane * step;
                     const bool below = pos < hi && __ldg(dl + pos) < lo_tok;
-                    const unsigned m = __ballot_sync(0xffffffffu, below);
-                    const int c = __popc(m);  // probes below lo_tok form a prefix
+                    const int c = __popc(__ballot_sync(0xffffffffu, below));
                     const int nlo = c > 0 ? lo + (c - 1) * step + 1 : lo;
                     const int nhi = min(hi, lo + c * step + (c < 32 ? 1 : 0));
                     lo = nlo;
@@ -396,7 +508,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 }
                 for (int base = lo;; base += 32) {
                     const int pos = base + lane;
-                    int v = pos < p.k ? __ldg(dl + pos) : INT32_MAX;
+                    const int v = pos < p.k ? __ldg(dl + pos) : INT32_MAX;
                     if (v <= hi_tok) {
                         const int tt = v / HW - x.t0, hh = (v / p.Wg) % p.Hg - x.h0,
                                   ww = v % p.Wg - x.w0;
@@ -408,174 +520,249 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ 
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&sh.flags_ready));
+            if (lane == 0) mbar_arrive(smem_addr(&sh.flags_full));
+            ++lc;
         }
+        if (!ok) fail();
     } else if (warp >= kWarpSoftmax0) {
-        // ------------------------------------------------------- softmax WGs
-        const int t = (warp - kWarpSoftmax0) >> 2;      // which query tile
+        // ============================================================ softmax WGs
+        const int t = (warp - kWarpSoftmax0) >> 2;                  // query tile slot
         const int r = threadIdx.x - (kWarpSoftmax0 + 4 * t) * 32;  // row in tile
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + (t == 0 ? C::kColS0 : C::kColS1);
         const uint32_t tO = tmem + lane_base + (t == 0 ? C::kColO0 : C::kColO1);
-        const int tile = t == 0 ? tile0 : tile1;
-
-        // ---- row identity and Q row load (into the K-major SW128 layout)
-        bool row_valid = false;
-        int token = 0;
-        int qs_t = 0, qs_h = 0, qs_w = 0;  // LOCAL: window starts of this row
-        Box bx;
-        if (MODE == DENSE) {
-            const int q = tile * kTileRows + r;
-            row_valid = tile < p.tiles && q < p.k;
-            if (row_valid) token = __ldg(p.dense_idx + (int64_t)b * p.k + q);
-        } else {
-            bx = local_box(p, tile);
-            const int qt = bx.t0 + r / (kBoxH * kBoxW), qh = bx.h0 + (r / kBoxW) % kBoxH,
-                      qw = bx.w0 + r % kBoxW;
-            row_valid = bx.active && qt < p.Tg && qh < p.Hg && qw < p.Wg;
-            token = (qt * p.Hg + qh) * p.Wg + qw;
-            qs_t = wstart(min(qt, p.Tg - 1), p.Tg, p.wt);
-            qs_h = wstart(min(qh, p.Hg - 1), p.Hg, p.wh);
-            qs_w = wstart(min(qw, p.Wg - 1), p.Wg, p.ww);
-        }
-        {
-            uint8_t *qt_smem = q_smem + t * C::kTileBytes;
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.Q + (bh * p.N + token) * D);
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
-                const uint4 v = row_valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-                const int sub = c >> 3, chunk = c & 7;
-                *reinterpret_cast<uint4 *>(qt_smem + sub * 16384 + r * 128 +
-                                           ((chunk ^ (r & 7)) << 4)) = v;
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(smem_addr(&sh.q_full[t]));
-        }
-
-        float m_run = -INFINITY, l = 0.f;
+        uint8_t *qt_smem = q_smem + t * C::kTileBytes;
+        uint32_t qi = 0, items = 0, sc = 0, lc = 0;
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            if (!mbar_wait(smem_addr(&sh.s_full[t]), (uint32_t)j & 1u, abort, kWaitLimitNs)) {
-                ok = false;
-                break;
+        while (ok) {
+            const int id = pop_item(qi++, ok);
+            if (!ok || id < 0) break;
+            const Item it = decode(p, id);
+            const bool dense = it.mode == DENSE;
+            const int tile = it.tile[t];
+            const int64_t row0 = (int64_t)it.bh * p.N;
+
+            // ---- row identity; DENSE rows are gathered into Q_t here
+            bool row_valid = false;
+            int token = 0, qs_t = 0, qs_h = 0, qs_w = 0;
+            Box bx;
+            if (dense) {
+                const int q = tile * kTileRows + r;
+                row_valid = tile < p.tiles_d && q < p.k;
+                if (row_valid) token = __ldg(p.dense_idx + (int64_t)it.b * p.k + q);
+                const uint4 *src = reinterpret_cast<const uint4 *>(p.Q + (row0 + token) * D);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 v = row_valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+                    const int sub = c >> 3, chunk = c & 7;
+                    *reinterpret_cast<uint4 *>(qt_smem + sub * 16384 + r * 128 +
+                                               ((chunk ^ (r & 7)) << 4)) = v;
+                }
+                fence_proxy_async_smem();
+                named_bar(1 + t, kTileRows);
+                if (r == 0) mbar_arrive(smem_addr(&sh.q_full[t]));
+            } else {
+                bx = local_box(p, tile);
+                const int qt = bx.t0 + r / (kBoxH * kBoxW), qh = bx.h0 + (r / kBoxW) % kBoxH,
+                          qw = bx.w0 + r % kBoxW;
+                row_valid = bx.active && qt < p.Tg && qh < p.Hg && qw < p.Wg;
+                token = (qt * p.Hg + qh) * p.Wg + qw;
+                qs_t = wstart(min(qt, p.Tg - 1), p.Tg, p.wt);
+                qs_h = wstart(min(qh, p.Hg - 1), p.Hg, p.wh);
+                qs_w = wstart(min(qw, p.Wg - 1), p.Wg, p.ww);
             }
-            tc_fence_after();
-            float sv[kTileKeys];
-            {
-                uint32_t raw[32];
+
+            float m_run = -INFINITY, l = 0.f;
+            for (int j = 0; j < it.n; ++j) {
+                if (!wait(sh.s_full[t], sc & 1u)) { ok = false; break; }
+                ++sc;
+                tc_fence_after();
+                float sv[kTileKeys];
 #pragma unroll
                 for (int c4 = 0; c4 < 4; ++c4) {
+                    uint32_t raw[32];
                     tmem_ld32(tS + 32 * c4, raw);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) sv[32 * c4 + i] = __uint_as_float(raw[i]);
                 }
-            }
-            // ---- mask
-            if (MODE == DENSE) {
-                const int valid = p.N - j * kTileKeys;
-                if (valid < kTileKeys) {
+                // ---- mask
+                if (dense) {
+                    const int valid = p.N - (it.kv_lo + j) * kTileKeys;
+                    if (valid < kTileKeys) {
 #pragma unroll
-                    for (int c = 0; c < kTileKeys; ++c)
-                        if (c >= valid) sv[c] = -INFINITY;
+                        for (int c = 0; c < kTileKeys; ++c)
+                            if (c >= valid) sv[c] = -INFINITY;
+                    }
+                } else {
+                    const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh, jw = j % p.nkw;
+                    const int kt = bx.tlo + jt, kh0 = bx.hlo + jh * kKvH, kw0 = bx.wlo + jw * kKvW;
+                    const bool t_ok = (unsigned)(kt - qs_t) < (unsigned)p.wt;
+                    const int wl = qs_w - kw0, whi = wl + p.ww;
+                    const uint32_t wbits =
+                        (whi <= 0 || wl >= kKvW)
+                            ? 0u
+                            : (((1u << min(whi, kKvW)) - 1u) & ~((1u << max(wl, 0)) - 1u));
+#pragma unroll
+                    for (int g = 0; g < kKvH; ++g) {
+                        const bool h_ok = t_ok && (unsigned)(kh0 + g - qs_h) < (unsigned)p.wh;
+                        const uint32_t bits = h_ok ? wbits : 0u;
+#pragma unroll
+                        for (int c = 0; c < kKvW; ++c)
+                            if (!((bits >> c) & 1u)) sv[g * kKvW + c] = -INFINITY;
+                    }
                 }
-            } else {
-                const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh, jw = j % p.nkw;
-                const int kt = bx.tlo + jt, kh0 = bx.hlo + jh * kKvH, kw0 = bx.wlo + jw * kKvW;
-                const bool t_ok = (unsigned)(kt - qs_t) < (unsigned)p.wt;
-                const int wl = qs_w - kw0, whi = wl + p.ww;
-                const uint32_t wbits =
-                    (whi <= 0 || wl >= kKvW)
-                        ? 0u
-                        : (((1u << min(whi, kKvW)) - 1u) & ~((1u << max(wl, 0)) - 1u));
+                // ---- online softmax (log2 domain)
+                float mt = sv[0];
 #pragma unroll
-                for (int g = 0; g < kKvH; ++g) {
-                    const bool h_ok = t_ok && (unsigned)(kh0 + g - qs_h) < (unsigned)p.wh;
-                    const uint32_t bits = h_ok ? wbits : 0u;
-#pragma unroll
-                    for (int c = 0; c < kKvW; ++c)
-                        if (!((bits >> c) & 1u)) sv[g * kKvW + c] = -INFINITY;
+                for (int c = 1; c < kTileKeys; ++c) mt = fmaxf(mt, sv[c]);
+                const float m_cand = fmaxf(m_run, mt * p.scale_log2);
+                const bool need = m_cand > m_run + kRescaleLog2;
+                float alpha = 1.f;
+                if (need) {
+                    alpha = ex2(m_run - m_cand);
+                    l *= alpha;
+                    m_run = m_cand;
                 }
-            }
-            // ---- online softmax (log2 domain)
-            float mt = sv[0];
+                if (j > 0 && __any_sync(0xffffffffu, need)) {
+                    // O_t holds P V of this item's tiles < j and no MMA writes it now
 #pragma unroll
-            for (int c = 1; c < kTileKeys; ++c) mt = fmaxf(mt, sv[c]);
-            const float m_cand = fmaxf(m_run, mt * p.scale_log2);
-            const bool need = m_cand > m_run + kRescaleLog2;
-            float alpha = 1.f;
-            if (need) {
-                alpha = ex2(m_run - m_cand);
-                l *= alpha;
-                m_run = m_cand;
+                    for (int c4 = 0; c4 < D / 32; ++c4) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + 32 * c4, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tO + 32 * c4, o);
+                    }
+                    tmem_wait_st();
+                }
+                const float m_use = m_run == -INFINITY ? 0.f : m_run;
+                float rs = 0.f;
+#pragma unroll
+                for (int c = 0; c < kTileKeys; ++c) {
+                    sv[c] = ex2(fmaf(sv[c], p.scale_log2, -m_use));
+                    rs += sv[c];
+                }
+                l += rs;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        pk[i] = pack_bf16(sv[64 * h2 + 2 * i], sv[64 * h2 + 2 * i + 1]);
+                    tmem_st32(tS + 32 * h2, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(smem_addr(&sh.p_full[t]));
             }
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                // O holds P V of tiles < j and no MMA writes it now
+            if (!ok) break;
+
+            // ---- epilogue: out row = O / l
+            if (!wait(sh.o_done[t], items & 1u)) { ok = false; break; }
+            tc_fence_after();
+            bool store = row_valid;
+            if (!dense) {
+                if (!wait(sh.flags_full, lc & 1u)) { ok = false; break; }
+                store = row_valid && !sh.no_store[t][r];
+                mbar_arrive(smem_addr(&sh.flags_empty));
+                ++lc;
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (row0 + token) * D);
+            if (dense && p.nsplit > 1) {
+                // ---- split key range: publish this partial; the last split merges
+                const int64_t prow =
+                    ((int64_t)(it.pair_id * p.nsplit + it.split) * 2 + t) * kTileRows + r;
+                float4 *po = reinterpret_cast<float4 *>(p.part_o + prow * D);
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t o[32];
                     tmem_ld32(tO + 32 * c4, o);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + 32 * c4, o);
+                    for (int v = 0; v < 8; ++v)
+                        __stcg(po + c4 * 8 + v,
+                               make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                           __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3])));
                 }
-                tmem_wait_st();
-            }
-            const float m_use = m_run == -INFINITY ? 0.f : m_run;
-            float rs = 0.f;
+                __stcg(p.part_ml + prow, make_float2(m_run, l));
+                __threadfence();
+                named_bar(1 + t, kTileRows);
+                if (r == 0) sh.fix_old[t] = atomicAdd(p.fix_count + it.pair_id * 2 + t, 1);
+                named_bar(1 + t, kTileRows);
+                const int old = *reinterpret_cast<volatile int *>(&sh.fix_old[t]);
+                if (old == p.nsplit - 1) {
+                    __threadfence();
+                    float mm = m_run;
+                    for (int sp = 0; sp < p.nsplit; ++sp) {
+                        if (sp == it.split) continue;
+                        const int64_t orow =
+                            ((int64_t)(it.pair_id * p.nsplit + sp) * 2 + t) * kTileRows + r;
+                        mm = fmaxf(mm, __ldcg(p.part_ml + orow).x);
+                    }
+                    float L = 0.f;
+                    for (int sp = 0; sp < p.nsplit; ++sp) {
+                        const int64_t orow =
+                            ((int64_t)(it.pair_id * p.nsplit + sp) * 2 + t) * kTileRows + r;
+                        const float2 ml = __ldcg(p.part_ml + orow);
+                        L += ml.y * ex2(ml.x - mm);
+                    }
+                    const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
-            for (int c = 0; c < kTileKeys; ++c) {
-                sv[c] = ex2(fmaf(sv[c], p.scale_log2, -m_use));
-                rs += sv[c];
-            }
-            l += rs;
+                    for (int c8 = 0; c8 < D / 8; ++c8) {
+                        float acc[8];
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t pk[32];
+                        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+                        for (int sp = 0; sp < p.nsplit; ++sp) {
+                            const int64_t orow =
+                                ((int64_t)(it.pair_id * p.nsplit + sp) * 2 + t) * kTileRows + r;
+                            const float a = ex2(__ldcg(p.part_ml + orow).x - mm);
+                            const float4 *src = reinterpret_cast<const float4 *>(p.part_o + orow * D);
+                            const float4 x0 = __ldcg(src + 2 * c8), x1 = __ldcg(src + 2 * c8 + 1);
+                            acc[0] += a * x0.x; acc[1] += a * x0.y; acc[2] += a * x0.z; acc[3] += a * x0.w;
+                            acc[4] += a * x1.x; acc[5] += a * x1.y; acc[6] += a * x1.z; acc[7] += a * x1.w;
+                        }
+                        if (store) {
+                            uint4 w;
+                            w.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+                            w.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+                            w.z = pack_bf16(acc[4] * inv, acc[5] * inv);
+                            w.w = pack_bf16(acc[6] * inv, acc[7] * inv);
+                            dst[c8] = w;
+                        }
+                    }
+                }
+            } else {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(sv[64 * h2 + 2 * i], sv[64 * h2 + 2 * i + 1]);
-                tmem_st32(tS + 32 * h2, pk);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(smem_addr(&sh.p_full[t]));
-        }
-        // ---- epilogue: out row = O / l
-        if (ok && !mbar_wait(smem_addr(&sh.o_done[t]), 0, abort, kWaitLimitNs)) ok = false;
-        bool store = ok && row_valid;
-        if (MODE == LOCAL && ok) {
-            if (!mbar_wait(smem_addr(&sh.flags_ready), 0, abort, kWaitLimitNs)) ok = false;
-            store = ok && row_valid && !sh.no_store[t][r];
-        }
-        if (!ok) fail();
-        tc_fence_after();
-        {
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (bh * p.N + token) * D);
+                for (int c4 = 0; c4 < D / 32; ++c4) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + 32 * c4, o);
+                    tmem_wait_ld();
+                    if (store) {
 #pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4) {
-                uint32_t o[32];
-                tmem_ld32(tO + 32 * c4, o);
-                tmem_wait_ld();
-                if (store) {
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv,
-                                        __uint_as_float(o[8 * v + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv,
-                                        __uint_as_float(o[8 * v + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv,
-                                        __uint_as_float(o[8 * v + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv,
-                                        __uint_as_float(o[8 * v + 7]) * inv);
-                        dst[c4 * 4 + v] = w;
+                        for (int v = 0; v < 4; ++v) {
+                            uint4 w;
+                            w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv,
+                                            __uint_as_float(o[8 * v + 1]) * inv);
+                            w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv,
+                                            __uint_as_float(o[8 * v + 3]) * inv);
+                            w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv,
+                                            __uint_as_float(o[8 * v + 5]) * inv);
+                            w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv,
+                                            __uint_as_float(o[8 * v + 7]) * inv);
+                            dst[c4 * 4 + v] = w;
+                        }
                     }
                 }
             }
+            tc_fence_before();
+            mbar_arrive(smem_addr(&sh.o_empty[t]));
+            ++items;
         }
+        if (!ok) fail();
     }
 
     tc_fence_before();
@@ -603,42 +790,80 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return fn;
 }
 
-// K or V viewed as [B*H][N][D] bf16; box = 128 keys x 64 channels.
-bool make_map_dense(CUtensorMap *m, const void *base, int BH, int N, int D)
+bool encode(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims,
+            const cuuint64_t *strides, const cuuint32_t *box)
 {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims, strides,
               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// K or V viewed as [B*H][T][H][W][D]; box = 1 x 8 x 16 keys x 64 channels.
-bool make_map_local(CUtensorMap *m, const void *base, int BH, int T, int Hg, int Wg, int D)
+// [B*H][N][D] bf16, box = 128 keys x 64 channels
+bool map_rows(CUtensorMap *m, const void *base, int BH, int N, int D)
 {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)T,
-                          (cuuint64_t)BH};
-    cuuint64_t strides[4] = {(cuuint64_t)D * 2, (cuuint64_t)Wg * D * 2,
-                             (cuuint64_t)Hg * Wg * D * 2, (cuuint64_t)T * Hg * Wg * D * 2};
-    cuuint32_t box[5] = {64, (cuuint32_t)kKvW, (cuuint32_t)kKvH, 1, 1};
-    cuuint32_t es[5] = {1, 1, 1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides,
-              box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)N * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kTileKeys, 1};
+    return encode(m, base, 3, dims, strides, box);
 }
 
-template <int D, int MODE>
-cudaError_t launch_mode(const AttnArgs &a, cudaStream_t s)
+// [B*H][T][H][W][D] bf16, box = bt x bh x bw tokens x 64 channels
+bool map_grid(CUtensorMap *m, const void *base, int BH, int T, int Hg, int Wg, int D, int bt,
+              int bh, int bw)
 {
-    using Cf = Cfg<D>;
+    const cuuint64_t dims[5] = {(cuuint64_t)D, (cuuint64_t)Wg, (cuuint64_t)Hg, (cuuint64_t)T,
+                                (cuuint64_t)BH};
+    const cuuint64_t strides[4] = {(cuuint64_t)D * 2, (cuuint64_t)Wg * D * 2,
+                                   (cuuint64_t)Hg * Wg * D * 2, (cuuint64_t)T * Hg * Wg * D * 2};
+    const cuuint32_t box[5] = {64, (cuuint32_t)bw, (cuuint32_t)bh, (cuuint32_t)bt, 1};
+    return encode(m, base, 5, dims, strides, box);
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
+                        int wh, int ww)
+{
+    AttnPlan pl;
+    pl.n_kv_d = (N + kTileKeys - 1) / kTileKeys;
+    pl.tiles_d = (k + kTileRows - 1) / kTileRows;
+    pl.pairs_d = (pl.tiles_d + 1) / 2;
+    const int64_t pairs_total = (int64_t)B * H * pl.pairs_d;
+    // split the key range in two when the dense pairs alone would not fill the SMs
+    // several times over; the LOCAL items then fill in behind the halves
+    pl.nsplit = (k > 0 && pairs_total < 4 * kPlanSMs && pl.n_kv_d >= 16) ? 2 : 1;
+    pl.kv_per_split = (pl.n_kv_d + pl.nsplit - 1) / pl.nsplit;
+    pl.n_dense_items = (int)(pairs_total * pl.nsplit);
+    const int nbt = (Tg + kBoxT - 1) / kBoxT;
+    pl.nbh = (Hg + kBoxH - 1) / kBoxH;
+    pl.nbw = (Wg + kBoxW - 1) / kBoxW;
+    pl.tiles_l = nbt * pl.nbh * pl.nbw;
+    pl.pairs_l = (pl.tiles_l + 1) / 2;
+    pl.nkt = min(kBoxT + wt - 1, Tg);
+    pl.nkh = (min(kBoxH + wh - 1, Hg) + kKvH - 1) / kKvH;
+    pl.nkw = (min(kBoxW + ww - 1, Wg) + kKvW - 1) / kKvW;
+    pl.n_kv_l = pl.nkt * pl.nkh * pl.nkw;
+    pl.n_local_items = k < N ? B * H * pl.pairs_l : 0;
+    pl.total_items = pl.n_dense_items + pl.n_local_items;
+    // workspace: counter | split arrivals | (m,l) partials | O partials
+    pl.off_fix = 256;
+    const size_t fix_bytes = pl.nsplit > 1 ? (size_t)pairs_total * 2 * sizeof(int) : 0;
+    pl.zero_bytes = pl.off_fix + fix_bytes;
+    pl.off_ml = align_up(pl.zero_bytes, 256);
+    const size_t rows = pl.nsplit > 1 ? (size_t)pairs_total * pl.nsplit * 2 * kTileRows : 0;
+    pl.off_o = align_up(pl.off_ml + rows * sizeof(float2), 256);
+    pl.workspace_bytes = pl.off_o + rows * d * sizeof(float);
+    return pl;
+}
+
+cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *workspace,
+                             cudaStream_t s)
+{
     Params p;
     p.Q = a.Q;
     p.out = a.out;
@@ -647,52 +872,44 @@ cudaError_t launch_mode(const AttnArgs &a, cudaStream_t s)
     p.B = a.B; p.H = a.H; p.N = a.N; p.k = a.k;
     p.Tg = a.Tg; p.Hg = a.Hg; p.Wg = a.Wg; p.wt = a.wt; p.wh = a.wh; p.ww = a.ww;
     p.scale_log2 = a.scale * 1.4426950408889634f;
-    CUtensorMap mk, mv;
-    if (MODE == DENSE) {
-        p.tiles = (a.k + kTileRows - 1) / kTileRows;
-        p.n_kv = (a.N + kTileKeys - 1) / kTileKeys;
-        p.nbh = p.nbw = p.nkt = p.nkh = p.nkw = 1;
-        if (!make_map_dense(&mk, a.K, a.B * a.H, a.N, D) ||
-            !make_map_dense(&mv, a.V, a.B * a.H, a.N, D))
-            return cudaErrorInvalidValue;
-    } else {
-        const int nbt = (a.Tg + kBoxT - 1) / kBoxT;
-        p.nbh = (a.Hg + kBoxH - 1) / kBoxH;
-        p.nbw = (a.Wg + kBoxW - 1) / kBoxW;
-        p.tiles = nbt * p.nbh * p.nbw;
-        p.nkt = min(kBoxT + a.wt - 1, a.Tg);
-        p.nkh = (min(kBoxH + a.wh - 1, a.Hg) + kKvH - 1) / kKvH;
-        p.nkw = (min(kBoxW + a.ww - 1, a.Wg) + kKvW - 1) / kKvW;
-        p.n_kv = p.nkt * p.nkh * p.nkw;
-        if (!make_map_local(&mk, a.K, a.B * a.H, a.Tg, a.Hg, a.Wg, D) ||
-            !make_map_local(&mv, a.V, a.B * a.H, a.Tg, a.Hg, a.Wg, D))
-            return cudaErrorInvalidValue;
-    }
-    auto kern = attn_tc_kernel<D, MODE>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cf::kSmem);
+    p.tiles_d = pl.tiles_d; p.pairs_d = pl.pairs_d; p.nsplit = pl.nsplit;
+    p.n_kv_d = pl.n_kv_d; p.kv_per_split = pl.kv_per_split; p.n_dense_items = pl.n_dense_items;
+    p.tiles_l = pl.tiles_l; p.pairs_l = pl.pairs_l; p.nbh = pl.nbh; p.nbw = pl.nbw;
+    p.nkt = pl.nkt; p.nkh = pl.nkh; p.nkw = pl.nkw; p.n_kv_l = pl.n_kv_l;
+    p.n_local_items = pl.n_local_items; p.total_items = pl.total_items;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    p.counter = reinterpret_cast<int *>(ws);
+    p.fix_count = reinterpret_cast<int *>(ws + pl.off_fix);
+    p.part_ml = reinterpret_cast<float2 *>(ws + pl.off_ml);
+    p.part_o = reinterpret_cast<float *>(ws + pl.off_o);
+    if (pl.total_items == 0) return cudaSuccess;
+
+    const int BH = a.B * a.H, D = a.d;
+    CUtensorMap k3, v3, k5, v5, q5;
+    if (!map_rows(&k3, a.K, BH, a.N, D) || !map_rows(&v3, a.V, BH, a.N, D) ||
+        !map_grid(&k5, a.K, BH, a.Tg, a.Hg, a.Wg, D, 1, kKvH, kKvW) ||
+        !map_grid(&v5, a.V, BH, a.Tg, a.Hg, a.Wg, D, 1, kKvH, kKvW) ||
+        !map_grid(&q5, a.Q, BH, a.Tg, a.Hg, a.Wg, D, kBoxT, kBoxH, kBoxW))
+        return cudaErrorInvalidValue;
+
+    cudaError_t e = cudaMemsetAsync(workspace, 0, pl.zero_bytes, s);
     if (e != cudaSuccess) return e;
-    dim3 grid((p.tiles + 1) / 2, a.H, a.B);
-    kern<<<grid, kThreads, Cf::kSmem, s>>>(mk, mv, p);
-    return cudaGetLastError();
-}
-
-template <int D>
-cudaError_t launch_d(const AttnArgs &a, cudaStream_t s)
-{
-    if (a.k < a.N) {
-        cudaError_t e = launch_mode<D, LOCAL>(a, s);
+    int dev = 0, sms = kPlanSMs;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = min(pl.total_items, sms);
+    if (D == 64) {
+        e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<64>::kSmem);
         if (e != cudaSuccess) return e;
+        attn_tc_kernel<64><<<grid, kThreads, Cfg<64>::kSmem, s>>>(k3, v3, k5, v5, q5, p);
+    } else {
+        e = cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Cfg<128>::kSmem);
+        if (e != cudaSuccess) return e;
+        attn_tc_kernel<128><<<grid, kThreads, Cfg<128>::kSmem, s>>>(k3, v3, k5, v5, q5, p);
     }
-    if (a.k > 0) return launch_mode<D, DENSE>(a, s);
-    return cudaSuccess;
-}
-
-}  // namespace
-
-cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s)
-{
-    return a.d == 64 ? launch_d<64>(a, s) : launch_d<128>(a, s);
+    return cudaGetLastError();
 }
 
 }  // namespace heta

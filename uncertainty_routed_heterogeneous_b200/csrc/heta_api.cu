@@ -27,7 +27,7 @@ const char *heta_status_string(int status)
     }
 }
 
-int heta_version(void) { return (1 << 16) | 0; }
+int heta_version(void) { return (1 << 16) | 1; }
 
 heta_status heta_dense_count(int N, double rho, int *k_out)
 {
@@ -57,31 +57,63 @@ heta_status heta_route(const float *u, int B, int N, int k, int32_t *dense_idx,
                                         static_cast<cudaStream_t>(stream)));
 }
 
-heta_status heta_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B,
-                           int H, int d, int Tg, int Hg, int Wg, int wt, int wh, int ww,
-                           float scale, const int32_t *dense_idx, int k, uint16_t *out,
-                           int32_t *status_dev, void *stream)
+}  // extern "C"
+
+namespace {
+
+heta_status check_attention_shape(int B, int H, int d, int Tg, int Hg, int Wg, int wt, int wh,
+                                  int ww, int k)
 {
     if (B < 1 || H < 1 || Tg < 1 || Hg < 1 || Wg < 1) return HETA_ERR_INVALID_ARG;
     const int64_t N64 = (int64_t)Tg * Hg * Wg;
     if (N64 >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
-    const int N = (int)N64;
-    if (k < 0 || k > N) return HETA_ERR_INVALID_ARG;
+    if (k < 0 || k > N64) return HETA_ERR_INVALID_ARG;
     if (wt < 1 || wh < 1 || ww < 1 || wt > Tg || wh > Hg || ww > Wg) return HETA_ERR_INVALID_ARG;
-    if (!(scale > 0.f) || !isfinite(scale)) return HETA_ERR_INVALID_ARG;
-    if (!Q || !K || !V || !out || (k > 0 && !dense_idx)) return HETA_ERR_INVALID_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
-        (dense_idx && !aligned16(dense_idx)))
-        return HETA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return HETA_ERR_UNSUPPORTED;
     if ((wt % 2) == 0 || (wh % 2) == 0 || (ww % 2) == 0) return HETA_ERR_UNSUPPORTED;
-    if ((int64_t)B * H * N * d >= (int64_t)1 << 40) return HETA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H * N64 * d >= (int64_t)1 << 40) return HETA_ERR_UNSUPPORTED;
+    if ((int64_t)B * H >= (int64_t)1 << 16) return HETA_ERR_UNSUPPORTED;
+    return HETA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg, int Wg, int wt,
+                                          int wh, int ww, int k, size_t *bytes)
+{
+    if (!bytes) return HETA_ERR_INVALID_ARG;
+    const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k);
+    if (st != HETA_OK) return st;
+    *bytes = heta::plan_attention(B, H, d, Tg * Hg * Wg, k, Tg, Hg, Wg, wt, wh, ww)
+                 .workspace_bytes;
+    return HETA_OK;
+}
+
+heta_status heta_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B,
+                           int H, int d, int Tg, int Hg, int Wg, int wt, int wh, int ww,
+                           float scale, const int32_t *dense_idx, int k, uint16_t *out,
+                           void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                           void *stream)
+{
+    const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k);
+    if (st != HETA_OK) return st;
+    const int N = Tg * Hg * Wg;
+    if (!(scale > 0.f) || !isfinite(scale)) return HETA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !out || (k > 0 && !dense_idx) || !workspace)
+        return HETA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
+        (dense_idx && !aligned16(dense_idx)) || !aligned16(workspace))
+        return HETA_ERR_INVALID_ARG;
+    const heta::AttnPlan plan = heta::plan_attention(B, H, d, N, k, Tg, Hg, Wg, wt, wh, ww);
+    if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
     heta::AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
     a.B = B; a.H = H; a.d = d; a.N = N; a.k = k;
     a.Tg = Tg; a.Hg = Hg; a.Wg = Wg; a.wt = wt; a.wh = wh; a.ww = ww;
     a.scale = scale;
-    return from_cuda(heta::launch_attention(a, static_cast<cudaStream_t>(stream)));
+    return from_cuda(heta::launch_attention(a, plan, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 heta_status heta_uncertainty(const uint16_t *X, const float *w, float bias, int B, int N,

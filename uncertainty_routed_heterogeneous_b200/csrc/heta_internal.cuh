@@ -35,6 +35,22 @@ struct AttnArgs {
     float scale;
 };
 
-cudaError_t launch_attention(const AttnArgs &a, cudaStream_t s);
+// How one heta_attention call is cut into work items, and its workspace.
+struct AttnPlan {
+    int tiles_d, pairs_d, n_kv_d, nsplit, kv_per_split, n_dense_items;
+    int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
+    int total_items;
+    size_t off_fix, off_ml, off_o, zero_bytes, workspace_bytes;
+};
+
+// SM count the work split is planned for (B200).  Only the balance depends
+// on it, never the result; the launch itself uses the device's real count.
+constexpr int kPlanSMs = 148;
+
+AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
+                        int wh, int ww);
+
+cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &plan, void *workspace,
+                             cudaStream_t s);
 
 }  // namespace heta
