@@ -41,7 +41,7 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kThreads = 384;           // 12 warps
+constexpr int kThreads = 384;           // 12 warps: one control and two softmax warpgroups
 constexpr int kTileRows = 128;          // query rows per tile (MMA M)
 constexpr int kTileKeys = 128;          // keys per K/V tile (MMA N of S)
 constexpr int kRingBytes = 128 * 1024;  // K/V ring
@@ -178,6 +178,96 @@ __device__ __forceinline__ Box local_box(const Params &p, int box)
     return x;
 }
 
+// One 128-key S tile of one query row (this thread's TMEM lane): mask, online
+// softmax update in the log2 domain, P = 2^(s*scale - m) in bf16 written over
+// the S columns it replaces, and the O rescale when the row maximum grew by
+// more than 2^8.  Reductions use 8 independent accumulators (one per group of
+// 16 columns) so no long dependency chain serialises the thread.  Groups
+// outside `active` (warp-uniform) are not read and get P = 0.
+// Masks: kAll -- every column is a key of the row; kPrefix -- columns below
+// `valid`; kWindow -- column 16g+c when bit g of hmask and bit c of wbits.
+enum { kAll = 0, kPrefix = 1, kWindow = 2 };
+
+template <int D, int MASK>
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_live, int valid,
+                                             uint32_t wbits, uint32_t hmask, uint32_t active,
+                                             float scale_log2, float &m_run, float &l)
+{
+    uint32_t sv[kTileKeys];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+        tmem_ld32(tS + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c4]));
+    tmem_wait_ld();
+    // column c of group g is a key of this row
+    auto key = [&](int g, int c) -> bool {
+        if (MASK == kPrefix) return 16 * g + c < valid;
+        if (MASK == kWindow) return ((hmask >> g) & (wbits >> c) & 1u) != 0u;
+        return true;
+    };
+    float mx[kKvH];
+#pragma unroll
+    for (int g = 0; g < kKvH; ++g) {
+        mx[g] = -INFINITY;
+        if (MASK == kAll || (active & (1u << g))) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const float x = __uint_as_float(sv[16 * g + c]);
+                mx[g] = fmaxf(mx[g], key(g, c) ? x : -INFINITY);
+            }
+        }
+    }
+    const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    const float m_cand = fmaxf(m_run, mt * scale_log2);
+    const bool need = m_cand > m_run + kRescaleLog2;
+    float alpha = 1.f;
+    if (need) {
+        alpha = ex2(m_run - m_cand);
+        l *= alpha;
+        m_run = m_cand;
+    }
+    const float m_use = m_run == -INFINITY ? 0.f : m_run;
+    float sm[kKvH];
+#pragma unroll
+    for (int g = 0; g < kKvH; ++g) {
+        sm[g] = 0.f;
+        if (MASK == kAll || (active & (1u << g))) {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                float e = ex2(fmaf(__uint_as_float(sv[16 * g + c]), scale_log2, -m_use));
+                if (MASK != kAll) e = key(g, c) ? e : 0.f;
+                sm[g] += e;
+                sv[16 * g + c] = __float_as_uint(e);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) sv[16 * g + c] = 0u;
+        }
+    }
+    l += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+    // bf16 pairs packed in place: word i <- columns 2i, 2i+1
+#pragma unroll
+    for (int i = 0; i < kTileKeys / 2; ++i)
+        sv[i] = pack_bf16(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+    tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+    tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+    tmem_wait_st();
+    if (o_live && __any_sync(0xffffffffu, need)) {
+        // O holds P V of the earlier tiles, and the next P V waits for this
+        // thread's p_full arrival: rescale it to the new maximum
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c4, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + 32 * c4, o);
+        }
+        tmem_wait_st();
+    }
+}
+
 struct Shared {
     uint64_t kv_full[16], kv_empty[16];
     uint64_t item_full[kQueue], item_empty[kQueue];
@@ -259,6 +349,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
         return id;
     };
 
+    // Registers: the control warpgroup gives up what the softmax warpgroups
+    // need for a full S row (4 x 56 + 8 x 224 = 12 x 168 per thread lane).
+    if (warp < kWarpSoftmax0) {
+    setmaxnreg_dec<56>();
     if (warp == kWarpTma) {
         // ============================================================ producer
         if (lane == 0) {
@@ -358,9 +452,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16(128, kTileKeys, false);
             const uint32_t id_o = idesc_bf16(128, D, true);
-            const uint32_t q_addr[2] = {smem_addr(q_smem), smem_addr(q_smem + C::kTileBytes)};
-            const uint32_t colS[2] = {C::kColS0, C::kColS1};
-            const uint32_t colO[2] = {C::kColO0, C::kColO1};
+            const uint32_t q_base = smem_addr(q_smem);
             uint32_t s = 0, qi = 0, items = 0;
             bool ok = true;
             auto wait_full = [&](uint32_t seq) -> uint32_t {
@@ -378,7 +470,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + colS[t], smem_desc_sw128(q_addr[t] + off, 16, 1024),
+                    mma_ss(tmem + (t ? C::kColS1 : C::kColS0),
+                           smem_desc_sw128(q_base + t * C::kTileBytes + off, 16, 1024),
                            smem_desc_sw128(k_addr + off, 16, 1024), id_s, kk > 0);
                 }
             };
@@ -386,7 +479,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             auto issue_pv = [&](int t, uint32_t v_addr, bool first) {
 #pragma unroll
                 for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-                    mma_ts(tmem + colO[t], tmem + colS[t] + kk * 8,
+                    mma_ts(tmem + (t ? C::kColO1 : C::kColO0), tmem + (t ? C::kColS1 : C::kColS0) + kk * 8,
                            smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), id_o,
                            (first && kk == 0) ? 0u : 1u);
                 }
@@ -524,10 +617,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             ++lc;
         }
         if (!ok) fail();
-    } else if (warp >= kWarpSoftmax0) {
+    }
+    } else {
         // ============================================================ softmax WGs
-        const int t = (warp - kWarpSoftmax0) >> 2;                  // query tile slot
-        const int r = threadIdx.x - (kWarpSoftmax0 + 4 * t) * 32;  // row in tile
+        setmaxnreg_inc<224>();
+        // a warp reaches TMEM lanes 32*(warp%4) .. +31: that quarter of the tile's rows
+        const int t = (warp - kWarpSoftmax0) >> 2;  // query tile slot
+        const int r = (warp & 3) * 32 + lane;       // row in tile
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + (t == 0 ? C::kColS0 : C::kColS1);
         const uint32_t tO = tmem + lane_base + (t == 0 ? C::kColO0 : C::kColO1);
@@ -577,84 +673,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 if (!wait(sh.s_full[t], sc & 1u)) { ok = false; break; }
                 ++sc;
                 tc_fence_after();
-                float sv[kTileKeys];
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    uint32_t raw[32];
-                    tmem_ld32(tS + 32 * c4, raw);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) sv[32 * c4 + i] = __uint_as_float(raw[i]);
-                }
-                // ---- mask
                 if (dense) {
                     const int valid = p.N - (it.kv_lo + j) * kTileKeys;
-                    if (valid < kTileKeys) {
-#pragma unroll
-                        for (int c = 0; c < kTileKeys; ++c)
-                            if (c >= valid) sv[c] = -INFINITY;
-                    }
+                    if (valid >= kTileKeys)
+                        softmax_tile<D, kAll>(tS, tO, j > 0, 0, 0u, 0u, 0xFFu, p.scale_log2,
+                                              m_run, l);
+                    else
+                        softmax_tile<D, kPrefix>(tS, tO, j > 0, valid, 0u, 0u, 0xFFu,
+                                                 p.scale_log2, m_run, l);
                 } else {
                     const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh, jw = j % p.nkw;
                     const int kt = bx.tlo + jt, kh0 = bx.hlo + jh * kKvH, kw0 = bx.wlo + jw * kKvW;
                     const bool t_ok = (unsigned)(kt - qs_t) < (unsigned)p.wt;
                     const int wl = qs_w - kw0, whi = wl + p.ww;
                     const uint32_t wbits =
-                        (whi <= 0 || wl >= kKvW)
+                        (!t_ok || whi <= 0 || wl >= kKvW)
                             ? 0u
                             : (((1u << min(whi, kKvW)) - 1u) & ~((1u << max(wl, 0)) - 1u));
+                    uint32_t hmask = 0;
 #pragma unroll
-                    for (int g = 0; g < kKvH; ++g) {
-                        const bool h_ok = t_ok && (unsigned)(kh0 + g - qs_h) < (unsigned)p.wh;
-                        const uint32_t bits = h_ok ? wbits : 0u;
-#pragma unroll
-                        for (int c = 0; c < kKvW; ++c)
-                            if (!((bits >> c) & 1u)) sv[g * kKvW + c] = -INFINITY;
-                    }
+                    for (int g = 0; g < kKvH; ++g)
+                        hmask |= ((unsigned)(kh0 + g - qs_h) < (unsigned)p.wh ? 1u : 0u) << g;
+                    // groups no row of this warp sees are skipped (their P is zero)
+                    const uint32_t active = __reduce_or_sync(0xffffffffu, wbits ? hmask : 0u);
+                    softmax_tile<D, kWindow>(tS, tO, j > 0, 0, wbits, hmask, active,
+                                             p.scale_log2, m_run, l);
                 }
-                // ---- online softmax (log2 domain)
-                float mt = sv[0];
-#pragma unroll
-                for (int c = 1; c < kTileKeys; ++c) mt = fmaxf(mt, sv[c]);
-                const float m_cand = fmaxf(m_run, mt * p.scale_log2);
-                const bool need = m_cand > m_run + kRescaleLog2;
-                float alpha = 1.f;
-                if (need) {
-                    alpha = ex2(m_run - m_cand);
-                    l *= alpha;
-                    m_run = m_cand;
-                }
-                if (j > 0 && __any_sync(0xffffffffu, need)) {
-                    // O_t holds P V of this item's tiles < j and no MMA writes it now
-#pragma unroll
-                    for (int c4 = 0; c4 < D / 32; ++c4) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + 32 * c4, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tO + 32 * c4, o);
-                    }
-                    tmem_wait_st();
-                }
-                const float m_use = m_run == -INFINITY ? 0.f : m_run;
-                float rs = 0.f;
-#pragma unroll
-                for (int c = 0; c < kTileKeys; ++c) {
-                    sv[c] = ex2(fmaf(sv[c], p.scale_log2, -m_use));
-                    rs += sv[c];
-                }
-                l += rs;
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        pk[i] = pack_bf16(sv[64 * h2 + 2 * i], sv[64 * h2 + 2 * i + 1]);
-                    tmem_st32(tS + 32 * h2, pk);
-                }
-                tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_addr(&sh.p_full[t]));
             }
