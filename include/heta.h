@@ -149,6 +149,34 @@ HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
                                     void *stream);
 
 /*
+ * heta_attention_noalloc -- heta_attention without a caller workspace.
+ *
+ * The paper has no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: code that must not call cudaMalloc (a
+ * real-time loop that may not block in the allocator, a host framework that
+ * owns every allocation, a context where allocation is not permitted).  It
+ * computes exactly what heta_attention computes, with the same arguments
+ * except the workspace, and allocates nothing.
+ *
+ * Its scratch is a fixed 16 MiB array in the library's device memory, which
+ * every GPU that loads the library keeps until the process exits.  Sizes
+ * whose scratch (heta_attention_workspace_size) exceeds 16 MiB are rejected
+ * with HETA_ERR_UNSUPPORTED before anything is launched; use heta_attention
+ * for those.  The first call on each device looks up the array's device
+ * address (a host-side runtime query, done once per device with that device
+ * current), so make the first call on a device before any stream capture.
+ * All calls share the array and it keeps the last call's contents; each call
+ * clears what must start at zero.  Calls whose kernels may overlap on the
+ * GPU (unordered streams) race on the array: order them.
+ */
+HETA_API heta_status heta_attention_noalloc(const uint16_t *Q, const uint16_t *K,
+                                            const uint16_t *V, int B, int H, int d,
+                                            int Tg, int Hg, int Wg, int wt, int wh, int ww,
+                                            float scale, const int32_t *dense_idx, int k,
+                                            uint16_t *out, int32_t *status_dev,
+                                            void *stream);
+
+/*
  * heta_uncertainty -- the lightweight per-token uncertainty head (Eq. (7)).
  *
  * u_out[b,i] = softplus(sum_c X[b,i,c] * w[c] + bias), softplus(z) =

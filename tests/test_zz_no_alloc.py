@@ -1,0 +1,79 @@
+"""heta_attention_noalloc: the allocation-free entry point.
+
+Some callers cannot allocate device memory (no cudaMalloc allowed where they
+run), so they cannot hand heta_attention a workspace.  heta_attention_noalloc
+takes the same arguments minus the workspace and keeps its scratch in a fixed
+16 MiB array inside the library.  This file checks, through the C ABI, that
+its output matches heta_attention's on two calls in a row (the second call
+reuses the array the first one left behind), and that sizes whose scratch
+would not fit are refused before anything runs.
+
+The file name sorts last so that a run stopping at the first failure has run
+every other test first.
+"""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+
+from helpers import MAX_ABS, MEAN_ABS, from_dev_bf16, to_dev, to_dev_bf16
+from uncertainty_routed_heterogeneous_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(lib):
+    fn = lib.heta_attention_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, vp] + [i] * 9 + [ctypes.c_float, vp, i, vp, vp, vp]
+    fn.restype = i
+    return fn
+
+
+@pytest.mark.parametrize("grid,win,rho,H,d", [
+    ((8, 16, 24), (3, 9, 9), 0.2, 2, 128),   # dense key range split in two
+    ((5, 12, 20), (3, 5, 7), 0.35, 3, 64),   # no split
+])
+def test_noalloc_matches_workspace_entry_point(gpu_lib, grid, win, rho, H, d):
+    import torch
+    heta = gpu_lib
+    lib = heta.load()
+    fn = _noalloc(lib)
+    w = W.scaled(W.WAN21, H=H, d=d, grid=grid, win=win, u_kind="uniform", u_seeds=(11,))
+    q, k, v = W.make_qkv(w)
+    Q, K, V = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+    kk = heta.dense_count(w.N, rho)
+    dense, _, _, _ = heta.route(to_dev(W.make_u(w)), kk)
+    ref = heta.attention(Q, K, V, w.grid, w.win, dense)
+    torch.cuda.synchronize()
+    want = from_dev_bf16(ref)
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for call in range(2):
+        out = torch.full_like(Q, float("nan"))
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        rc = fn(ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(K.data_ptr()),
+                ctypes.c_void_p(V.data_ptr()), w.B, w.H, w.d, grid[0], grid[1], grid[2],
+                win[0], win[1], win[2], ctypes.c_float(1.0 / math.sqrt(d)),
+                ctypes.c_void_p(dense.data_ptr()), kk, ctypes.c_void_p(out.data_ptr()),
+                ctypes.c_void_p(st.data_ptr()), stream)
+        assert rc == heta.HETA_OK, heta.status_string(rc)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        got = from_dev_bf16(out)
+        assert np.all(np.isfinite(got)), "call %d left rows unwritten" % call
+        err = np.abs(got - want)
+        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (call, err.max(), err.mean())
+
+
+def test_noalloc_refuses_sizes_beyond_its_array(gpu_lib):
+    """The Wan2.1-shaped call at rho = 0.2 needs ~83 MB of scratch: refused up front."""
+    heta = gpu_lib
+    fn = _noalloc(heta.load())
+    k = heta.dense_count(32760, 0.2)
+    need = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k)
+    assert need > 16 << 20
+    fake = ctypes.c_void_p(1 << 20)
+    rc = fn(fake, fake, fake, 1, 12, 128, 21, 30, 52, 3, 9, 9, ctypes.c_float(0.088), fake, k,
+            fake, None, None)
+    assert rc == heta.HETA_ERR_UNSUPPORTED

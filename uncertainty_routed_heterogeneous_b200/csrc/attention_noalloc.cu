@@ -1,0 +1,73 @@
+// attention_noalloc.cu -- heta_attention for callers that cannot allocate.
+//
+// heta_attention needs device scratch (the work-item counter of the
+// persistent kernel and, when the dense rows' key range is split, the halves'
+// partial results).  Some callers cannot provide it: code that must not call
+// cudaMalloc at all (a real-time loop that may not block on the allocator, a
+// plug-in host that owns every allocation, code running where the allocator
+// is off limits).  heta_attention_noalloc runs the same kernel with its
+// scratch in a fixed array that lives in this file's device memory.
+//
+// The array is kStaticScratchBytes (16 MiB) and every GPU that loads the
+// library keeps it until the process exits.  Calls share it and it keeps the
+// previous call's contents: each call clears the counters it needs before its
+// kernel runs, and two calls whose kernels overlap on the GPU (different
+// streams, no ordering between them) race on it.
+#include <mutex>
+
+#include "heta_internal.cuh"
+
+namespace heta {
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(16) << 20;
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices];  // device address of the array, per device
+
+// Device address of the array on the current device.  In host code the
+// array's name is only a stand-in, so the address is looked up once per
+// device (with that device current) and remembered.
+cudaError_t scratch_on_current_device(void **ptr)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *ptr = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace heta
+
+extern "C" {
+
+HETA_API heta_status heta_attention_noalloc(const uint16_t *Q, const uint16_t *K,
+                                            const uint16_t *V, int B, int H, int d, int Tg,
+                                            int Hg, int Wg, int wt, int wh, int ww, float scale,
+                                            const int32_t *dense_idx, int k, uint16_t *out,
+                                            int32_t *status_dev, void *stream)
+{
+    size_t need = 0;
+    heta_status st =
+        heta_attention_workspace_size(B, H, d, Tg, Hg, Wg, wt, wh, ww, k, &need);
+    if (st != HETA_OK) return st;
+    if (need > heta::kStaticScratchBytes) return HETA_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if (heta::scratch_on_current_device(&scratch) != cudaSuccess) return HETA_ERR_CUDA;
+    return heta_attention(Q, K, V, B, H, d, Tg, Hg, Wg, wt, wh, ww, scale, dense_idx, k, out,
+                          scratch, heta::kStaticScratchBytes, status_dev, stream);
+}
+
+}  // extern "C"
