@@ -465,24 +465,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 return smem_addr(ring + (size_t)stage * C::kTileBytes);
             };
             auto release = [&](uint32_t seq) { mma_commit(smem_addr(&sh.kv_empty[seq % C::kStages])); };
-            // S_t = Q_t K^T : M=128, N=128 keys, K=D (both operands K-major)
             auto issue_s = [&](int t, uint32_t k_addr) {
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    mma_ss(tmem + (t ? C::kColS1 : C::kColS0),
-                           smem_desc_sw128(q_base + t * C::kTileBytes + off, 16, 1024),
-                           smem_desc_sw128(k_addr + off, 16, 1024), id_s, kk > 0);
-                }
+                const uint64_t qd = smem_desc_sw128(q_base + t * C::kTileBytes, 16, 1024);
+                const uint64_t kd = smem_desc_sw128(k_addr, 16, 1024);
+                if (D == 128)
+                    mma_ss_k128<16384, 16384>(tmem + (t ? C::kColS1 : C::kColS0), qd, kd, id_s, 0u);
+                else
+                    mma_ss_k64(tmem + (t ? C::kColS1 : C::kColS0), qd, kd, id_s, 0u);
             };
-            // O_t += P_t V : M=128, N=D, K=128 keys; P from TMEM, V MN-major
             auto issue_pv = [&](int t, uint32_t v_addr, bool first) {
-#pragma unroll
-                for (int kk = 0; kk < kTileKeys / 16; ++kk) {
-                    mma_ts(tmem + (t ? C::kColO1 : C::kColO0), tmem + (t ? C::kColS1 : C::kColS0) + kk * 8,
-                           smem_desc_sw128(v_addr + kk * 2048, 16384, 1024), id_o,
-                           (first && kk == 0) ? 0u : 1u);
-                }
+                mma_ts_steps<8, 2048>(tmem + (t ? C::kColO1 : C::kColO0),
+                                      tmem + (t ? C::kColS1 : C::kColS0),
+                                      smem_desc_sw128(v_addr, 16384, 1024), id_o, first ? 0u : 1u);
             };
             uint32_t pc[2] = {0, 0};  // p_full phases consumed per slot
             while (ok) {
