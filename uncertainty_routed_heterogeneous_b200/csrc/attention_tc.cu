@@ -474,7 +474,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                     mma_ss_k64(tmem + (t ? C::kColS1 : C::kColS0), qd, kd, id_s, 0u);
             };
             auto issue_pv = [&](int t, uint32_t v_addr, bool first) {
-                mma_ts_steps<8, 2048>(tmem + (t ? C::kColO1 : C::kColO0),
+                mma_ts_k128<2048>(tmem + (t ? C::kColO1 : C::kColO0),
                                       tmem + (t ? C::kColS1 : C::kColS0),
                                       smem_desc_sw128(v_addr, 16384, 1024), id_o, first ? 0u : 1u);
             };

@@ -182,23 +182,32 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 
 // D (+)= A * B^T over K = 128 as eight K=16 MMAs, A and B both K-major,
 // 128-byte swizzled in shared memory; the 64-column halves of A and B start
-// A_SUB and B_SUB bytes after the first.  One asm block: two adds per MMA.
+// A_SUB and B_SUB bytes after the first.  All eight descriptor pairs are
+// formed first (independent adds), then the eight MMAs issue back to back.
 template <int A_SUB, int B_SUB>
 __device__ __forceinline__ void mma_ss_k128(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t"
+        "{\n\t.reg .pred p, t;\n\t"
+        ".reg .b64 a1, a2, a3, a4, a5, a6, a7, b1, b2, b3, b4, b5, b6, b7;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "setp.eq.u32 t, 0, 0;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 b1, %2, 2;\n\t"
+        "add.s64 a2, %1, 4;\n\tadd.s64 b2, %2, 4;\n\t"
+        "add.s64 a3, %1, 6;\n\tadd.s64 b3, %2, 6;\n\t"
+        "add.s64 a4, %1, %5;\n\tadd.s64 b4, %2, %6;\n\t"
+        "add.s64 a5, %1, %7;\n\tadd.s64 b5, %2, %8;\n\t"
+        "add.s64 a6, %1, %9;\n\tadd.s64 b6, %2, %10;\n\t"
+        "add.s64 a7, %1, %11;\n\tadd.s64 b7, %2, %12;\n\t"
         HETA_MMA_F16 "[%0], %1, %2, %3, p;\n\t"
-        "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, %5;\n\tadd.s64 b, %2, %6;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %8;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, %9;\n\tadd.s64 b, %2, %10;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, %11;\n\tadd.s64 b, %2, %12;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t}"
+        HETA_MMA_F16 "[%0], a1, b1, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a2, b2, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a3, b3, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a4, b4, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a5, b5, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a6, b6, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a7, b7, %3, t;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate),
         "n"(A_SUB / 16), "n"(B_SUB / 16), "n"(A_SUB / 16 + 2), "n"(B_SUB / 16 + 2),
         "n"(A_SUB / 16 + 4), "n"(B_SUB / 16 + 4), "n"(A_SUB / 16 + 6), "n"(B_SUB / 16 + 6)
@@ -210,55 +219,51 @@ __device__ __forceinline__ void mma_ss_k64(uint32_t d_tmem, uint64_t a_desc, uin
                                            uint32_t idesc, uint32_t accumulate)
 {
     asm volatile(
-        "{\n\t.reg .pred p, t;\n\t.reg .b64 a, b;\n\t"
+        "{\n\t.reg .pred p, t;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "setp.eq.u32 t, 0, 0;\n\t"
+        "add.s64 a1, %1, 2;\n\tadd.s64 b1, %2, 2;\n\t"
+        "add.s64 a2, %1, 4;\n\tadd.s64 b2, %2, 4;\n\t"
+        "add.s64 a3, %1, 6;\n\tadd.s64 b3, %2, 6;\n\t"
         HETA_MMA_F16 "[%0], %1, %2, %3, p;\n\t"
-        "add.s64 a, %1, 2;\n\tadd.s64 b, %2, 2;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, 4;\n\tadd.s64 b, %2, 4;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t"
-        "add.s64 a, %1, 6;\n\tadd.s64 b, %2, 6;\n\t" HETA_MMA_F16 "[%0], a, b, %3, t;\n\t}"
+        HETA_MMA_F16 "[%0], a1, b1, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a2, b2, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], a3, b3, %3, t;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
 // D (+)= A * B with A (bf16 pairs) in TMEM and B MN-major in shared memory:
-// NK K=16 MMAs; step kk reads A columns a_tmem + 8kk and B rows 16kk..16kk+15
-// (B_STEP bytes further on).
-template <int NK, int B_STEP>
-__device__ __forceinline__ void mma_ts_steps(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                             uint32_t idesc, uint32_t accumulate)
+// eight K=16 MMAs; step kk reads A columns a_tmem + 8kk and B rows
+// 16kk..16kk+15 (kk * B_STEP bytes further on).
+template <int B_STEP>
+__device__ __forceinline__ void mma_ts_k128(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate)
 {
-    static_assert(NK == 4 || NK == 8, "4 or 8 K-steps");
-    if (NK == 4) {
-        asm volatile(
-            "{\n\t.reg .pred p, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-            "setp.ne.b32 p, %4, 0;\n\t"
-            "setp.eq.u32 t, 0, 0;\n\t"
-            HETA_MMA_F16 "[%0], [%1], %2, %3, p;\n\t"
-            "add.u32 a, %1, 8;\n\tadd.s64 b, %2, %5;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 16;\n\tadd.s64 b, %2, %6;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 24;\n\tadd.s64 b, %2, %7;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t}"
-            ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate),
-            "n"(B_STEP / 16), "n"(2 * B_STEP / 16), "n"(3 * B_STEP / 16)
-            : "memory");
-    } else {
-        asm volatile(
-            "{\n\t.reg .pred p, t;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-            "setp.ne.b32 p, %4, 0;\n\t"
-            "setp.eq.u32 t, 0, 0;\n\t"
-            HETA_MMA_F16 "[%0], [%1], %2, %3, p;\n\t"
-            "add.u32 a, %1, 8;\n\tadd.s64 b, %2, %5;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 16;\n\tadd.s64 b, %2, %6;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 24;\n\tadd.s64 b, %2, %7;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 32;\n\tadd.s64 b, %2, %8;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 40;\n\tadd.s64 b, %2, %9;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 48;\n\tadd.s64 b, %2, %10;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t"
-            "add.u32 a, %1, 56;\n\tadd.s64 b, %2, %11;\n\t" HETA_MMA_F16 "[%0], [a], b, %3, t;\n\t}"
-            ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate),
-            "n"(B_STEP / 16), "n"(2 * B_STEP / 16), "n"(3 * B_STEP / 16), "n"(4 * B_STEP / 16),
-            "n"(5 * B_STEP / 16), "n"(6 * B_STEP / 16), "n"(7 * B_STEP / 16)
-            : "memory");
-    }
+    asm volatile(
+        "{\n\t.reg .pred p, t;\n\t"
+        ".reg .b64 b1, b2, b3, b4, b5, b6, b7;\n\t.reg .b32 a1, a2, a3, a4, a5, a6, a7;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.u32 t, 0, 0;\n\t"
+        "add.u32 a1, %1, 8;\n\tadd.s64 b1, %2, %5;\n\t"
+        "add.u32 a2, %1, 16;\n\tadd.s64 b2, %2, %6;\n\t"
+        "add.u32 a3, %1, 24;\n\tadd.s64 b3, %2, %7;\n\t"
+        "add.u32 a4, %1, 32;\n\tadd.s64 b4, %2, %8;\n\t"
+        "add.u32 a5, %1, 40;\n\tadd.s64 b5, %2, %9;\n\t"
+        "add.u32 a6, %1, 48;\n\tadd.s64 b6, %2, %10;\n\t"
+        "add.u32 a7, %1, 56;\n\tadd.s64 b7, %2, %11;\n\t"
+        HETA_MMA_F16 "[%0], [%1], %2, %3, p;\n\t"
+        HETA_MMA_F16 "[%0], [a1], b1, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], [a2], b2, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], [a3], b3, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], [a4], b4, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], [a5], b5, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], [a6], b6, %3, t;\n\t"
+        HETA_MMA_F16 "[%0], [a7], b7, %3, t;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate),
+        "n"(B_STEP / 16), "n"(2 * B_STEP / 16), "n"(3 * B_STEP / 16), "n"(4 * B_STEP / 16),
+        "n"(5 * B_STEP / 16), "n"(6 * B_STEP / 16), "n"(7 * B_STEP / 16)
+        : "memory");
 }
 
 // Arrives once on the mbarrier when every MMA issued so far by this thread is done.
