@@ -215,6 +215,28 @@ def cpu_baseline(args, w):
             "sample": s.describe(), "seconds": dt}
 
 
+def profiled_traffic(workload_name):
+    """DRAM bytes per launch of attn_tc_kernel from the committed ncu summary --
+    only when that summary covers this workload and was taken on the current
+    kernel source (else None)."""
+    import hashlib
+    import re
+    if workload_name != W.WAN21.name:
+        return None
+    src = os.path.join(ROOT, "uncertainty_routed_heterogeneous_b200", "csrc", "attention_tc.cu")
+    prof = os.path.join(ROOT, "profiles", "attn_tc_kernel-wan2.1-1.3b-rho0.2.md")
+    try:
+        text = open(prof).read()
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    m = re.search(r"source_sha256_16: (\w+)", text)
+    b = re.search(r"dram_bytes_per_launch: (\d+)", text)
+    if m and b and m.group(1) == sha:
+        return int(b.group(1))
+    return None
+
+
 def config_of(w, n_gpus):
     k = math.ceil(round(w.rho * w.N, 9))
     return {"workload": w.name, "B": w.B, "H": w.H, "d": w.d,
@@ -382,7 +404,8 @@ def run_heta(args, info):
                      "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                      "frac": tflops / peak, "frac_of_burst": tflops / peaks["bf16_tflops"],
                      "peak_source": "%s sustained bf16 (cuBLAS)" % peaks["source"],
-                     "traffic": None, "algorithmic_flops": flops},
+                     "traffic": profiled_traffic(base.name), "traffic_unit": "bytes/launch",
+                     "algorithmic_flops": flops},
         "head_roofline": {"bound": "hbm",
                           "achieved": (w.B * w.N * w.C * 2 + w.C * 4 + w.B * w.N * 4) /
                           (head_ms * 1e6),
