@@ -185,34 +185,35 @@ __device__ __forceinline__ Box local_box(const Params &p, int box)
 // 16 columns) so no long dependency chain serialises the thread.  Groups
 // outside `active` (warp-uniform) are not read and get P = 0.
 // Masks: kAll -- every column is a key of the row; kPrefix -- columns below
-// `valid`; kWindow -- column 16g+c when bit g of hmask and bit c of wbits.
+// `valid`; kWindow -- column c of group g when bit g of gmask is set and
+// wbias[c] is 0 (wbias[c] = -inf marks a column outside the row's window).
+// Masked scores become -inf in the max pass, so the exp pass needs no mask.
 enum { kAll = 0, kPrefix = 1, kWindow = 2 };
 
 template <int D, int MASK>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_live, int valid,
-                                             uint32_t wbits, uint32_t hmask, uint32_t active,
-                                             float scale_log2, float &m_run, float &l)
+                                             const float (&wbias)[kKvW], uint32_t gmask,
+                                             uint32_t active, float scale_log2, float &m_run,
+                                             float &l)
 {
     uint32_t sv[kTileKeys];
 #pragma unroll
     for (int c4 = 0; c4 < 4; ++c4)
         tmem_ld32(tS + 32 * c4, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c4]));
     tmem_wait_ld();
-    // column c of group g is a key of this row
-    auto key = [&](int g, int c) -> bool {
-        if (MASK == kPrefix) return 16 * g + c < valid;
-        if (MASK == kWindow) return ((hmask >> g) & (wbits >> c) & 1u) != 0u;
-        return true;
-    };
     float mx[kKvH];
 #pragma unroll
     for (int g = 0; g < kKvH; ++g) {
         mx[g] = -INFINITY;
-        if (MASK == kAll || (active & (1u << g))) {
+        if (MASK != kWindow || (active & (1u << g))) {
+            const bool gv = (gmask >> g) & 1u;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                const float x = __uint_as_float(sv[16 * g + c]);
-                mx[g] = fmaxf(mx[g], key(g, c) ? x : -INFINITY);
+                float x = __uint_as_float(sv[16 * g + c]);
+                if (MASK == kPrefix) x = 16 * g + c < valid ? x : -INFINITY;
+                if (MASK == kWindow) x = gv ? x + wbias[c] : -INFINITY;
+                if (MASK != kAll) sv[16 * g + c] = __float_as_uint(x);
+                mx[g] = fmaxf(mx[g], x);
             }
         }
     }
@@ -231,11 +232,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_li
 #pragma unroll
     for (int g = 0; g < kKvH; ++g) {
         sm[g] = 0.f;
-        if (MASK == kAll || (active & (1u << g))) {
+        if (MASK != kWindow || (active & (1u << g))) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                float e = ex2(fmaf(__uint_as_float(sv[16 * g + c]), scale_log2, -m_use));
-                if (MASK != kAll) e = key(g, c) ? e : 0.f;
+                const float e = ex2(fmaf(__uint_as_float(sv[16 * g + c]), scale_log2, -m_use));
                 sm[g] += e;
                 sv[16 * g + c] = __float_as_uint(e);
             }
@@ -663,6 +663,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             }
 
             float m_run = -INFINITY, l = 0.f;
+            float wbias[kKvW];           // LOCAL: 0 / -inf per column of the current w range
+            int wbias_w0 = -(1 << 30);   // w of the first column wbias was built for
+#pragma unroll
+            for (int c = 0; c < kKvW; ++c) wbias[c] = 0.f;
             for (int j = 0; j < it.n; ++j) {
                 if (!wait(sh.s_full[t], sc & 1u)) { ok = false; break; }
                 ++sc;
@@ -670,27 +674,29 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 if (dense) {
                     const int valid = p.N - (it.kv_lo + j) * kTileKeys;
                     if (valid >= kTileKeys)
-                        softmax_tile<D, kAll>(tS, tO, j > 0, 0, 0u, 0u, 0xFFu, p.scale_log2,
+                        softmax_tile<D, kAll>(tS, tO, j > 0, 0, wbias, 0u, 0xFFu, p.scale_log2,
                                               m_run, l);
                     else
-                        softmax_tile<D, kPrefix>(tS, tO, j > 0, valid, 0u, 0u, 0xFFu,
+                        softmax_tile<D, kPrefix>(tS, tO, j > 0, valid, wbias, 0u, 0xFFu,
                                                  p.scale_log2, m_run, l);
                 } else {
                     const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh, jw = j % p.nkw;
                     const int kt = bx.tlo + jt, kh0 = bx.hlo + jh * kKvH, kw0 = bx.wlo + jw * kKvW;
+                    if (kw0 != wbias_w0) {
+                        // columns kw0 .. kw0+15 inside the row's w-window get bias 0
+                        wbias_w0 = kw0;
+#pragma unroll
+                        for (int c = 0; c < kKvW; ++c)
+                            wbias[c] = (unsigned)(kw0 + c - qs_w) < (unsigned)p.ww ? 0.f : -INFINITY;
+                    }
                     const bool t_ok = (unsigned)(kt - qs_t) < (unsigned)p.wt;
-                    const int wl = qs_w - kw0, whi = wl + p.ww;
-                    const uint32_t wbits =
-                        (!t_ok || whi <= 0 || wl >= kKvW)
-                            ? 0u
-                            : (((1u << min(whi, kKvW)) - 1u) & ~((1u << max(wl, 0)) - 1u));
-                    uint32_t hmask = 0;
+                    uint32_t gmask = 0;
 #pragma unroll
                     for (int g = 0; g < kKvH; ++g)
-                        hmask |= ((unsigned)(kh0 + g - qs_h) < (unsigned)p.wh ? 1u : 0u) << g;
+                        gmask |= (t_ok && (unsigned)(kh0 + g - qs_h) < (unsigned)p.wh ? 1u : 0u) << g;
                     // groups no row of this warp sees are skipped (their P is zero)
-                    const uint32_t active = __reduce_or_sync(0xffffffffu, wbits ? hmask : 0u);
-                    softmax_tile<D, kWindow>(tS, tO, j > 0, 0, wbits, hmask, active,
+                    const uint32_t active = __reduce_or_sync(0xffffffffu, gmask);
+                    softmax_tile<D, kWindow>(tS, tO, j > 0, 0, wbias, gmask, active,
                                              p.scale_log2, m_run, l);
                 }
                 tc_fence_before();
