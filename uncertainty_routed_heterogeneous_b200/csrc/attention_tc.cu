@@ -109,6 +109,33 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
+// Two fp32 lanes in one 64-bit register (low = first), for the packed f32x2 ops.
+__device__ __forceinline__ uint64_t f2(uint32_t lo_bits, uint32_t hi_bits)
+{
+    return ((uint64_t)hi_bits << 32) | lo_bits;
+}
+
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 __device__ __forceinline__ void named_bar(int id, int nthreads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -208,17 +235,26 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_li
         if (MASK != kWindow || (active & (1u << g))) {
             const bool gv = (gmask >> g) & 1u;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                float x = __uint_as_float(sv[16 * g + c]);
-                if (MASK == kPrefix) x = 16 * g + c < valid ? x : -INFINITY;
-                if (MASK == kWindow) x = gv ? x + wbias[c] : -INFINITY;
-                if (MASK != kAll) sv[16 * g + c] = __float_as_uint(x);
-                mx[g] = fmaxf(mx[g], x);
+            for (int c = 0; c < 16; c += 2) {
+                float x0 = __uint_as_float(sv[16 * g + c]);
+                float x1 = __uint_as_float(sv[16 * g + c + 1]);
+                if (MASK == kPrefix) {
+                    x0 = 16 * g + c < valid ? x0 : -INFINITY;
+                    x1 = 16 * g + c + 1 < valid ? x1 : -INFINITY;
+                }
+                if (MASK == kWindow) {
+                    x0 = gv ? x0 + wbias[c] : -INFINITY;
+                    x1 = gv ? x1 + wbias[c + 1] : -INFINITY;
+                }
+                if (MASK != kAll) {
+                    sv[16 * g + c] = __float_as_uint(x0);
+                    sv[16 * g + c + 1] = __float_as_uint(x1);
+                }
+                mx[g] = max3(mx[g], x0, x1);
             }
         }
     }
-    const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    const float mt = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
     const float m_cand = fmaxf(m_run, mt * scale_log2);
     const bool need = m_cand > m_run + kRescaleLog2;
     float alpha = 1.f;
@@ -228,27 +264,32 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_li
         m_run = m_cand;
     }
     const float m_use = m_run == -INFINITY ? 0.f : m_run;
-    float sm[kKvH];
+    // P in column pairs: x = s*scale - m as one packed fp32 FMA, 2^x of each,
+    // the pair added to one of four packed fp32 sums, and the bf16 pair word
+    // i <- columns 2i, 2i+1 written in place (sv[i] after sv[2i], sv[2i+1] are read)
+    const uint64_t scale2 = f2(__float_as_uint(scale_log2), __float_as_uint(scale_log2));
+    const uint64_t negm2 = f2(__float_as_uint(-m_use), __float_as_uint(-m_use));
+    uint64_t sum2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int g = 0; g < kKvH; ++g) {
-        sm[g] = 0.f;
         if (MASK != kWindow || (active & (1u << g))) {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float e = ex2(fmaf(__uint_as_float(sv[16 * g + c]), scale_log2, -m_use));
-                sm[g] += e;
-                sv[16 * g + c] = __float_as_uint(e);
+            for (int c = 0; c < 16; c += 2) {
+                const uint64_t x2 = fma_f32x2(f2(sv[16 * g + c], sv[16 * g + c + 1]), scale2, negm2);
+                const float e0 = ex2(__uint_as_float((uint32_t)x2));
+                const float e1 = ex2(__uint_as_float((uint32_t)(x2 >> 32)));
+                sum2[g & 3] = add_f32x2(sum2[g & 3], f2(__float_as_uint(e0), __float_as_uint(e1)));
+                sv[8 * g + c / 2] = pack_bf16(e0, e1);
             }
         } else {
 #pragma unroll
-            for (int c = 0; c < 16; ++c) sv[16 * g + c] = 0u;
+            for (int c = 0; c < 16; c += 2) sv[8 * g + c / 2] = 0u;
         }
     }
-    l += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
-    // bf16 pairs packed in place: word i <- columns 2i, 2i+1
-#pragma unroll
-    for (int i = 0; i < kTileKeys / 2; ++i)
-        sv[i] = pack_bf16(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
+    l += ((__uint_as_float((uint32_t)sum2[0]) + __uint_as_float((uint32_t)(sum2[0] >> 32))) +
+          (__uint_as_float((uint32_t)sum2[1]) + __uint_as_float((uint32_t)(sum2[1] >> 32)))) +
+         ((__uint_as_float((uint32_t)sum2[2]) + __uint_as_float((uint32_t)(sum2[2] >> 32))) +
+          (__uint_as_float((uint32_t)sum2[3]) + __uint_as_float((uint32_t)(sum2[3] >> 32))));
     tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
     tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
     tmem_wait_st();
