@@ -212,14 +212,14 @@ __device__ __forceinline__ Box local_box(const Params &p, int box)
 // 16 columns) so no long dependency chain serialises the thread.  Groups
 // outside `active` (warp-uniform) are not read and get P = 0.
 // Masks: kAll -- every column is a key of the row; kPrefix -- columns below
-// `valid`; kWindow -- column c of group g when bit g of gmask is set and
-// wbias[c] is 0 (wbias[c] = -inf marks a column outside the row's window).
+// `valid`; kWindow -- column c of group g when bit g of gmask is set and the
+// column's entry in wbias2 is 0 (-inf marks a column outside the row's window).
 // Masked scores become -inf in the max pass, so the exp pass needs no mask.
 enum { kAll = 0, kPrefix = 1, kWindow = 2 };
 
 template <int D, int MASK>
 __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_live, int valid,
-                                             const float (&wbias)[kKvW], uint32_t gmask,
+                                             const uint64_t (&wbias2)[kKvW / 2], uint32_t gmask,
                                              uint32_t active, float scale_log2, float &m_run,
                                              float &l)
 {
@@ -233,7 +233,9 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_li
     for (int g = 0; g < kKvH; ++g) {
         mx[g] = -INFINITY;
         if (MASK != kWindow || (active & (1u << g))) {
-            const bool gv = (gmask >> g) & 1u;
+            // kWindow: + 0 / -inf for the column, then + 0 / -inf for the group (row h)
+            const uint32_t gb = ((gmask >> g) & 1u) ? 0u : 0xff800000u;
+            const uint64_t gb2 = f2(gb, gb);
 #pragma unroll
             for (int c = 0; c < 16; c += 2) {
                 float x0 = __uint_as_float(sv[16 * g + c]);
@@ -243,8 +245,12 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool o_li
                     x1 = 16 * g + c + 1 < valid ? x1 : -INFINITY;
                 }
                 if (MASK == kWindow) {
-                    x0 = gv ? x0 + wbias[c] : -INFINITY;
-                    x1 = gv ? x1 + wbias[c + 1] : -INFINITY;
+                    const uint64_t x2 =
+                        add_f32x2(add_f32x2(f2(__float_as_uint(x0), __float_as_uint(x1)),
+                                            wbias2[c / 2]),
+                                  gb2);
+                    x0 = __uint_as_float((uint32_t)x2);
+                    x1 = __uint_as_float((uint32_t)(x2 >> 32));
                 }
                 if (MASK != kAll) {
                     sv[16 * g + c] = __float_as_uint(x0);
@@ -704,10 +710,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             }
 
             float m_run = -INFINITY, l = 0.f;
-            float wbias[kKvW];           // LOCAL: 0 / -inf per column of the current w range
-            int wbias_w0 = -(1 << 30);   // w of the first column wbias was built for
+            uint64_t wbias2[kKvW / 2];   // LOCAL: 0 / -inf per column of the current w range, paired
+            int wbias_w0 = -(1 << 30);   // w of the first column wbias2 was built for
 #pragma unroll
-            for (int c = 0; c < kKvW; ++c) wbias[c] = 0.f;
+            for (int c = 0; c < kKvW / 2; ++c) wbias2[c] = 0ull;
             for (int j = 0; j < it.n; ++j) {
                 if (!wait(sh.s_full[t], sc & 1u)) { ok = false; break; }
                 ++sc;
@@ -715,10 +721,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 if (dense) {
                     const int valid = p.N - (it.kv_lo + j) * kTileKeys;
                     if (valid >= kTileKeys)
-                        softmax_tile<D, kAll>(tS, tO, j > 0, 0, wbias, 0u, 0xFFu, p.scale_log2,
+                        softmax_tile<D, kAll>(tS, tO, j > 0, 0, wbias2, 0u, 0xFFu, p.scale_log2,
                                               m_run, l);
                     else
-                        softmax_tile<D, kPrefix>(tS, tO, j > 0, valid, wbias, 0u, 0xFFu,
+                        softmax_tile<D, kPrefix>(tS, tO, j > 0, valid, wbias2, 0u, 0xFFu,
                                                  p.scale_log2, m_run, l);
                 } else {
                     const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh, jw = j % p.nkw;
@@ -727,8 +733,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                         // columns kw0 .. kw0+15 inside the row's w-window get bias 0
                         wbias_w0 = kw0;
 #pragma unroll
-                        for (int c = 0; c < kKvW; ++c)
-                            wbias[c] = (unsigned)(kw0 + c - qs_w) < (unsigned)p.ww ? 0.f : -INFINITY;
+                        for (int c = 0; c < kKvW; c += 2)
+                            wbias2[c / 2] = f2((unsigned)(kw0 + c - qs_w) < (unsigned)p.ww ? 0u : 0xff800000u,
+                                               (unsigned)(kw0 + c + 1 - qs_w) < (unsigned)p.ww ? 0u : 0xff800000u);
                     }
                     const bool t_ok = (unsigned)(kt - qs_t) < (unsigned)p.wt;
                     uint32_t gmask = 0;
@@ -737,7 +744,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                         gmask |= (t_ok && (unsigned)(kh0 + g - qs_h) < (unsigned)p.wh ? 1u : 0u) << g;
                     // groups no row of this warp sees are skipped (their P is zero)
                     const uint32_t active = __reduce_or_sync(0xffffffffu, gmask);
-                    softmax_tile<D, kWindow>(tS, tO, j > 0, 0, wbias, gmask, active,
+                    softmax_tile<D, kWindow>(tS, tO, j > 0, 0, wbias2, gmask, active,
                                              p.scale_log2, m_run, l);
                 }
                 tc_fence_before();
