@@ -563,10 +563,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                     const bool last = j + 1 == n;
                     uint32_t v_addr = 0, kn_addr = 0, v_seq = 0, kn_seq = 0;
                     for (int t = 0; t < 2 && ok; ++t) {
+                        // the tiles this slot needs next are waited for first: they
+                        // usually landed long ago, and the softmax is usually later
                         if (!dense || t == 0) {
                             v_seq = s++;
                             v_addr = wait_full(v_seq);
                             if (!ok) break;
+                            if (!last) {
+                                kn_seq = s++;
+                                kn_addr = wait_full(kn_seq);
+                                if (!ok) break;
+                            }
                         }
                         if (!wait(sh.p_full[t], pc[t] & 1u)) { ok = false; break; }
                         ++pc[t];
@@ -578,20 +585,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                         }
                         tc_fence_after();
                         issue_pv(t, v_addr, j == 0);
-                        if (!dense || t == 1) release(v_seq);
                         if (last) {
                             mma_commit(smem_addr(&sh.o_done[t]));
-                            continue;
+                        } else {
+                            issue_s(t, kn_addr);
+                            mma_commit(smem_addr(&sh.s_full[t]));
+                            if (j + 2 == n) mma_commit(smem_addr(&sh.q_empty[t]));
                         }
-                        if (!dense || t == 0) {
-                            kn_seq = s++;
-                            kn_addr = wait_full(kn_seq);
-                            if (!ok) break;
+                        if (!dense || t == 1) {
+                            release(v_seq);
+                            if (!last) release(kn_seq);
                         }
-                        issue_s(t, kn_addr);
-                        mma_commit(smem_addr(&sh.s_full[t]));
-                        if (!dense || t == 1) release(kn_seq);
-                        if (j + 2 == n) mma_commit(smem_addr(&sh.q_empty[t]));
                     }
                 }
                 ++items;
