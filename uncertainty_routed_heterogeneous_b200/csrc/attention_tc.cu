@@ -357,9 +357,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             mbar_init(smem_addr(&sh.q_full[t]), 1);
             mbar_init(smem_addr(&sh.q_empty[t]), 1);
             mbar_init(smem_addr(&sh.s_full[t]), 1);
-            mbar_init(smem_addr(&sh.p_full[t]), kTileRows);
+            mbar_init(smem_addr(&sh.p_full[t]), kTileRows / 32);  // one arrival per warp
             mbar_init(smem_addr(&sh.o_done[t]), 1);
-            mbar_init(smem_addr(&sh.o_empty[t]), kTileRows);
+            mbar_init(smem_addr(&sh.o_empty[t]), kTileRows / 32);
         }
         mbar_init(smem_addr(&sh.flags_full), 1);
         mbar_init(smem_addr(&sh.flags_empty), 2 * kTileRows);
@@ -752,7 +752,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                                              p.scale_log2, m_run, l);
                 }
                 tc_fence_before();
-                mbar_arrive(smem_addr(&sh.p_full[t]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&sh.p_full[t]));
             }
             if (!ok) break;
 
@@ -855,7 +856,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_addr(&sh.o_empty[t]));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&sh.o_empty[t]));
             ++items;
         }
         if (!ok) fail();
