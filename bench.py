@@ -53,6 +53,10 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense-compare", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-window-sweep", action="store_true",
+                   help="skip timing the 9^3 / 11^3 / 13^3 windows of the paper's ablation")
+    p.add_argument("--cpu-seconds", type=float, default=10.0,
+                   help="minimum host time the cpu_baseline oracle sample runs for")
     return p.parse_args()
 
 
@@ -205,14 +209,20 @@ def run_reference(args, info):
 
 
 def cpu_baseline(args, w):
+    """The oracle on repeated token samples until at least --cpu-seconds have passed."""
     import oracle
     s = OracleSample(w, n_tokens=args.cpu_tokens)
     s.step()  # warm: page in, build
     t0 = time.perf_counter()
-    n = s.step()
-    dt = time.perf_counter() - t0
+    n = reps = 0
+    while True:
+        n += s.step()
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= args.cpu_seconds:
+            break
     return {"value": n / dt, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": s.describe(), "seconds": dt}
+            "sample": "%d repetitions of: %s" % (reps, s.describe()), "seconds": dt}
 
 
 def profiled_traffic(workload_name):
@@ -352,6 +362,30 @@ def run_heta(args, info):
         dense_cmp = {"ms": full_ms, "tflops": full_flops / (full_ms * 1e9),
                      "speedup_of_routed": full_ms / attn_ms}
 
+    # ---- the paper's window ablation sizes (Table 7) on the same inputs -------
+    win_sweep = None
+    if not args.no_window_sweep:
+        win_sweep = {}
+        for n in W.WINDOW_CUBES:
+            wn = W.window_cube(n)
+            ws_n = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, wn.win, kk),
+                               dtype=torch.uint8, device=dev)
+            heta.attention(d_Q, d_K, d_V, w.grid, wn.win, dense, out=out, workspace=ws_n)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            e0.record()
+            for _ in range(reps):
+                heta.attention(d_Q, d_K, d_V, w.grid, wn.win, dense, out=out, workspace=ws_n)
+            e1.record()
+            torch.cuda.synchronize()
+            ms_n = e0.elapsed_time(e1) / reps
+            fl_n = heta.attention_flops(w.B, w.H, w.d, w.N, kk, wn.M)
+            win_sweep["x".join(map(str, wn.win))] = {
+                "attention_ms": ms_n, "algorithmic_tflops": fl_n / (ms_n * 1e9),
+                "speedup_vs_dense": (dense_cmp["ms"] / ms_n) if dense_cmp else None}
+        del ws_n
+
     # ---- end to end through the public API with host buffers ----------------
     e2e = None
     if not args.no_e2e:
@@ -411,6 +445,7 @@ def run_heta(args, info):
                           (head_ms * 1e6),
                           "peak": peaks["hbm_gbs"], "unit": "GB/s"},
         "dense_compare": dense_cmp,
+        "window_sweep": win_sweep,
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu, "clocks": sampler.summary(),
     }

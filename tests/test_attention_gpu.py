@@ -87,3 +87,20 @@ def test_rho1_equals_dense_and_rho0_equals_local(gpu_lib):
     a = run(gpu_lib, w, rho=1.0)
     b = run(gpu_lib, w, rho=0.0)
     assert a and b
+
+
+# The paper's window ablation (Table 7): 9^3, 11^3 (its default) and 13^3
+# neighbourhoods.  All rows on a grid just large enough for 13 along every
+# axis (ragged tiles everywhere), then sampled rows at the Wan2.1 shape.
+@pytest.mark.parametrize("n", W.WINDOW_CUBES)
+@pytest.mark.parametrize("rho", [0.0, 0.2])
+def test_window_cube_all_rows(gpu_lib, n, rho):
+    w = dataclasses.replace(W.scaled(W.WAN21, H=2, grid=(13, 17, 27), win=(n, n, n),
+                                     u_kind="uniform", u_seeds=(12,)),
+                            name="window%d-13x17x27" % n)
+    run(gpu_lib, w, rho=rho)
+
+
+@pytest.mark.parametrize("n", W.WINDOW_CUBES)
+def test_window_cube_full_size_sampled_rows(gpu_lib, n):
+    run(gpu_lib, W.window_cube(n), n_sample=1000)

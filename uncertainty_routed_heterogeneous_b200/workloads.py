@@ -72,6 +72,15 @@ def sweep(rho: float, u_kind: str) -> Workload:
 
 ALL = {w.name: w for w in (TINY, WAN21, WAN22, BATCHED)}
 
+# the window sizes the paper's window ablation compares (its default 11^3,
+# plus 9^3 and 13^3), at the Wan2.1 latent shape
+WINDOW_CUBES = (9, 11, 13)
+
+
+def window_cube(n: int) -> Workload:
+    """The Wan2.1 workload with an n x n x n local window."""
+    return replace(WAN21, name="wan2.1-1.3b-window%d" % n, win=(n, n, n))
+
 
 def scaled(w: Workload, **kw) -> Workload:
     """A smaller copy of a workload (for tests that must finish in seconds)."""
