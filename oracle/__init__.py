@@ -40,6 +40,8 @@ def _load():
         lib.oracle_route.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
                                      ctypes.c_void_p]
+        lib.oracle_route_threshold.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_double] + [ctypes.c_void_p] * 5
         lib.oracle_window_start.argtypes = [ctypes.c_int] * 3
         lib.oracle_window.argtypes = [ctypes.c_int] * 7 + [ctypes.c_void_p]
         lib.oracle_attention_rows.argtypes = (
@@ -93,6 +95,28 @@ def route(u: np.ndarray, k: int):
     if rc:
         raise OracleError(rc)
     return dense, local, mask
+
+
+def route_threshold(u: np.ndarray, c: float):
+    """Routing by the paper's threshold T = mu + c*sigma (Eq. (11)-(12), reading R8).
+
+    u: [B,N] float32.  Returns (counts [B], dense_idx [B,N], local_idx [B,N],
+    thresh [B] float64, mask [B,N]); row b of dense_idx holds counts[b]
+    ascending token ids (the rest is padding), row b of local_idx the other
+    N - counts[b]; mask is m_i (1 = local).
+    """
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    B, N = u.shape
+    counts = np.zeros(B, np.int32)
+    dense = np.full((B, N), -1, np.int32)
+    local = np.full((B, N), -1, np.int32)
+    thresh = np.zeros(B, np.float64)
+    mask = np.zeros((B, N), np.uint8)
+    rc = _load().oracle_route_threshold(_ptr(u), B, N, float(c), _ptr(counts), _ptr(dense),
+                                        _ptr(local), _ptr(thresh), _ptr(mask))
+    if rc:
+        raise OracleError(rc)
+    return counts, dense, local, thresh, mask
 
 
 def window_start(p: int, extent: int, width: int) -> int:

@@ -36,6 +36,10 @@
  *   R7 the uncertainty head is u = softplus(x . w + b).  The paper names it
  *      only as a "lightweight branch" with u >= 0; a linear map followed by
  *      softplus is the plainest form that satisfies Eq. (7).
+ *   R8 threshold mode (the paper's own rule): mu and sigma are the mean and
+ *      the population standard deviation of one sample's N uncertainties,
+ *      in fp64; u == T goes dense (Eq. (12)'s strict "<").  The count then
+ *      varies per sample.
  *
  * All arithmetic is IEEE fp64 on inputs that are exactly representable
  * (fp32 arrays holding bf16 values, or fp32 values), in plain loop order.
@@ -109,6 +113,51 @@ int oracle_route(const float *u, int B, int N, int k,
     }
     free(order);
     free(is_dense);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Routing by the paper's own threshold rule, Eq. (11)-(12) (R8).      */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Per sample b: mu = (1/N) sum_i u_i and sigma = sqrt((1/N) sum_i (u_i - mu)^2)
+ * (the population standard deviation, two passes), T = mu + c * sigma
+ * (Eq. (11)), m_i = [u_i < T] (Eq. (12)): u_i >= T goes dense.  All in fp64,
+ * summed in index order.  Writes counts[b] = |dense set|, dense_idx row b
+ * (capacity N: entries 0..counts[b]-1, ascending), local_idx row b (entries
+ * 0..N-counts[b]-1, ascending), thresh[b] = T (optional) and mask (optional,
+ * 1 = local).  N = 0 gives empty sets; a NaN in u is status 4.
+ */
+int oracle_route_threshold(const float *u, int B, int N, double c, int32_t *counts,
+                           int32_t *dense_idx, int32_t *local_idx, double *thresh,
+                           uint8_t *mask)
+{
+    if (B < 0 || N < 0 || isnan(c) || isinf(c)) return ORACLE_INVALID;
+    for (int64_t i = 0; i < (int64_t)B * N; ++i)
+        if (isnan(u[i])) return ORACLE_NONFINITE;
+    for (int b = 0; b < B; ++b) {
+        const float *ub = u + (int64_t)b * N;
+        double sum = 0.0;
+        for (int i = 0; i < N; ++i) sum += (double)ub[i];
+        const double mu = N > 0 ? sum / (double)N : 0.0;
+        double sq = 0.0;
+        for (int i = 0; i < N; ++i) {
+            const double dev = (double)ub[i] - mu;
+            sq += dev * dev;
+        }
+        const double sigma = N > 0 ? sqrt(sq / (double)N) : 0.0;
+        const double T = mu + c * sigma;
+        if (thresh) thresh[b] = T;
+        int nd = 0, nl = 0;
+        for (int i = 0; i < N; ++i) {
+            const int local = (double)ub[i] < T;
+            if (local) local_idx[(int64_t)b * N + nl++] = i;
+            else dense_idx[(int64_t)b * N + nd++] = i;
+            if (mask) mask[(int64_t)b * N + i] = (uint8_t)local;
+        }
+        counts[b] = nd;
+    }
     return ORACLE_OK;
 }
 

@@ -13,6 +13,9 @@ What pins what:
   * route        -- hand-worked tie cases (golden/route_ties.txt), Python's own
                     sort on (-u, i), and the complete characterisation of a
                     top-k set with index tie-break
+  * threshold    -- hand-worked mu + c*sigma cases (golden/route_threshold.txt),
+                    numpy's mean/std (ddof=0) in fp64, the Gaussian tail
+                    fraction 1 - Phi(c), shift/scale invariance, u == T dense
   * attention    -- torch's scaled_dot_product_attention in fp64 (a library
                     routine) with no mask (rho = 1) and with a boolean window
                     mask built from the independent window definition (rho=0);
@@ -245,6 +248,118 @@ def test_route_nan_is_an_error():
     with pytest.raises(oracle.OracleError) as e:
         oracle.route(u, 1)
     assert e.value.code == oracle.NONFINITE
+
+
+# --------------------------------------------------------------------------
+# threshold routing, the paper's own rule (Eq. (11)-(12), reading R8)
+# --------------------------------------------------------------------------
+
+def read_threshold_golden():
+    """golden/route_threshold.txt: u values | c | T | dense ids (worked by hand)."""
+    cases = []
+    for line in open(os.path.join(GOLDEN, "route_threshold.txt")):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        u, c, T, dense = (f.strip() for f in line.split("|"))
+        cases.append((np.array([[float(x) for x in u.split()]], np.float32), float(c),
+                      float(T), [int(x) for x in dense.split()] if dense else []))
+    return cases
+
+
+@pytest.mark.parametrize("case", read_threshold_golden())
+def test_threshold_golden(case):
+    u, c, T, dense = case
+    counts, d, l, thresh, mask = oracle.route_threshold(u, c)
+    assert abs(thresh[0] - T) <= 1e-6 * max(1.0, abs(T))
+    assert counts[0] == len(dense)
+    assert d[0, :counts[0]].tolist() == dense
+    N = u.shape[1]
+    assert sorted(d[0, :counts[0]].tolist() + l[0, :N - counts[0]].tolist()) == list(range(N))
+    assert all(mask[0, i] == (0 if i in dense else 1) for i in range(N))
+
+
+def _numpy_threshold_sets(u, c):
+    """Independent restatement with numpy's own mean and std in fp64."""
+    T = np.mean(u.astype(np.float64), axis=1) + c * np.std(u.astype(np.float64), axis=1, ddof=0)
+    return T, u.astype(np.float64) >= T[:, None]
+
+
+@pytest.mark.parametrize("c", [-0.5, 0.0, 0.9, 2.0])
+@pytest.mark.parametrize("kind", ["gauss", "uniform", "smooth"])
+def test_threshold_vs_numpy(c, kind):
+    rng = np.random.default_rng(7)
+    B, N = 3, 4099
+    if kind == "gauss":
+        u = rng.standard_normal((B, N)).astype(np.float32)
+    elif kind == "uniform":
+        u = rng.random((B, N), dtype=np.float32)
+    else:
+        u = np.stack([W.make_u(W.scaled(W.WAN21, grid=(3, 29, 47), u_seeds=(s,)))[0]
+                      for s in (1, 2, 3)])
+        B, N = u.shape
+    counts, d, l, thresh, mask = oracle.route_threshold(u, c)
+    T, dense = _numpy_threshold_sets(u, c)
+    assert np.allclose(thresh, T, rtol=1e-12, atol=1e-12)
+    for b in range(B):
+        want = np.nonzero(dense[b])[0]
+        # decisions are only uncertain inside the rounding band of T
+        band = np.abs(u[b].astype(np.float64) - T[b]) <= 1e-9 * max(1.0, abs(T[b]))
+        got = d[b, :counts[b]]
+        assert np.array_equal(np.setdiff1d(got, np.nonzero(band)[0]),
+                              np.setdiff1d(want, np.nonzero(band)[0]))
+        assert np.array_equal(l[b, :N - counts[b]], np.setdiff1d(np.arange(N), got))
+        assert np.array_equal(mask[b] == 0, np.isin(np.arange(N), got))
+
+
+def test_threshold_gaussian_tail_fraction():
+    """c = 0.9 on Gaussian u keeps 1 - Phi(0.9) = 0.184 of the tokens dense
+    (the paper's rho ~ 0.2 setting), c = 0 half of them."""
+    rng = np.random.default_rng(11)
+    u = rng.standard_normal((4, 32760)).astype(np.float32)
+    for c in (0.0, 0.9, 1.5):
+        counts = oracle.route_threshold(u, c)[0]
+        tail = 0.5 * math.erfc(c / math.sqrt(2.0))
+        # binomial std at N = 32760 is < 0.003; the estimated mu/sigma add less
+        assert np.all(np.abs(counts / 32760.0 - tail) < 0.012), (c, counts)
+
+
+def test_threshold_shift_and_scale_invariant():
+    """T moves with an affine map a*u + b (a > 0) and the sets do not change.
+    Values on a 1/8 grid keep every step exact in fp32 and fp64."""
+    rng = np.random.default_rng(5)
+    u = (rng.integers(-64, 64, size=(2, 3001)) / 8.0).astype(np.float32)
+    base = oracle.route_threshold(u, 0.7)
+    for a, b in ((4.0, 0.0), (1.0, 96.0), (0.5, -3.0)):
+        v = (u * np.float32(a) + np.float32(b)).astype(np.float32)
+        got = oracle.route_threshold(v, 0.7)
+        assert np.array_equal(got[0], base[0])
+        assert np.array_equal(got[1], base[1])
+        assert np.allclose(got[3], a * base[3] + b, rtol=1e-12)
+
+
+def test_threshold_constant_u_is_all_dense():
+    """sigma = 0 puts T on every u; u == T goes dense (Eq. (12)'s strict <)."""
+    u = np.full((2, 777), 0.3125, np.float32)
+    counts, d, l, thresh, mask = oracle.route_threshold(u, 1.0)
+    assert counts.tolist() == [777, 777]
+    assert np.all(thresh == 0.3125)
+    assert not mask.any()
+
+
+def test_threshold_edge_cases():
+    empty = np.zeros((2, 0), np.float32)
+    counts = oracle.route_threshold(empty, 0.9)[0]
+    assert counts.tolist() == [0, 0]
+    with pytest.raises(oracle.OracleError) as e:
+        oracle.route_threshold(np.array([[0.1, float("nan")]], np.float32), 0.0)
+    assert e.value.code == oracle.NONFINITE
+    # samples are routed independently
+    u = np.stack([np.arange(10, dtype=np.float32), -np.arange(10, dtype=np.float32)])
+    counts, d, _, thresh, _ = oracle.route_threshold(u, 0.0)
+    assert counts.tolist() == [5, 5]
+    assert d[0, :5].tolist() == [5, 6, 7, 8, 9] and d[1, :5].tolist() == [0, 1, 2, 3, 4]
+    assert thresh.tolist() == [4.5, -4.5]
 
 
 # --------------------------------------------------------------------------
