@@ -96,6 +96,38 @@ HETA_API heta_status heta_route(const float *u, int B, int N, int k,
                        int32_t *status_dev, void *stream);
 
 /*
+ * heta_route_threshold -- routing by the paper's own rule (Eq. (11)-(12)):
+ * per sample b, T_b = mu_b + c * sigma_b, where mu_b and sigma_b are the mean
+ * and the population standard deviation of u[b,:], computed in fp64; token i
+ * is dense when u[b,i] >= T_b (m_i = [u_i < T] of Eq. (12)), compared in
+ * fp64.  The dense count therefore varies per sample.  Smaller c routes more
+ * tokens to dense attention (c = 0.9 keeps about 18% of Gaussian u dense).
+ * A NaN in u raises status_dev to HETA_ERR_NONFINITE (outputs unspecified).
+ *
+ *   u          [B,N] fp32, read only.
+ *   c          finite.
+ *   counts     [B] int32 out (device): |D_b|.
+ *   dense_idx  [B,N] int32 out: row b holds D_b in increasing token order in
+ *              entries 0..counts[b]-1; the rest of the row is not written.
+ *   local_idx  [B,N] int32 out: row b holds the complement, increasing, in
+ *              entries 0..N-counts[b]-1; the rest is not written.
+ *   thresh_out [B] fp64 out, or NULL: T_b.
+ *   mask_out   [B,N] uint8 out, or NULL: m_i, 1 = local, 0 = dense.
+ *   status_dev device int32, or NULL.
+ *
+ * The sums run in a fixed order, so repeated calls give identical results;
+ * a u within a few fp64 ulps of T may fall on either side compared with
+ * another summation order.  Same size limits as heta_route; pointers
+ * 16-byte aligned; one CTA per sample.  heta_attention_counts consumes the
+ * outputs without a round trip to the host.
+ */
+HETA_API heta_status heta_route_threshold(const float *u, int B, int N, double c,
+                                          int32_t *counts, int32_t *dense_idx,
+                                          int32_t *local_idx, double *thresh_out,
+                                          uint8_t *mask_out, int32_t *status_dev,
+                                          void *stream);
+
+/*
  * heta_attention_workspace_size -- device scratch one heta_attention call
  * needs for these sizes (host-only; touches no device).
  *
@@ -147,6 +179,30 @@ HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
                                     uint16_t *out, void *workspace,
                                     size_t workspace_bytes, int32_t *status_dev,
                                     void *stream);
+
+/*
+ * heta_attention_counts -- heta_attention with a per-sample dense count that
+ * lives on the device (the heta_route_threshold output), so no count has to
+ * come back to the host first.
+ *
+ *   dense_idx  [B,k_cap] int32: row b holds D_b, strictly increasing, in
+ *              entries 0..counts[b]-1 (row stride k_cap; the rest of the row
+ *              is not read).  heta_route_threshold writes k_cap = N rows.
+ *   counts     [B] int32 (device): |D_b|; values outside 0..k_cap are
+ *              clamped to it.
+ *   workspace  at least heta_attention_workspace_size(..., k = k_cap) bytes.
+ *
+ * Every other argument, requirement and error is as for heta_attention with
+ * k = k_cap.  The work is planned for k_cap dense rows per sample; work
+ * items past a sample's count end at once, so a generous k_cap costs little.
+ */
+HETA_API heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K,
+                                           const uint16_t *V, int B, int H, int d, int Tg,
+                                           int Hg, int Wg, int wt, int wh, int ww, float scale,
+                                           const int32_t *dense_idx, int k_cap,
+                                           const int32_t *counts, uint16_t *out,
+                                           void *workspace, size_t workspace_bytes,
+                                           int32_t *status_dev, void *stream);
 
 /*
  * heta_attention_noalloc -- heta_attention without a caller workspace.

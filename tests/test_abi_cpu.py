@@ -34,7 +34,8 @@ def declared_symbols():
 def test_header_declares_the_three_path_calls():
     names = declared_symbols()
     assert {"heta_route", "heta_attention", "heta_uncertainty", "heta_dense_count",
-            "heta_status_string", "heta_version", "heta_attention_workspace_size"} <= names
+            "heta_status_string", "heta_version", "heta_attention_workspace_size",
+            "heta_route_threshold", "heta_attention_counts"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -99,6 +100,40 @@ def test_host_validation_returns_before_any_launch(lib):
         heta.HETA_ERR_INVALID_ARG
     assert lib.heta_uncertainty(fake, fake, ctypes.c_float(0.0), 1, 10, 32768, fake, N, N) == \
         heta.HETA_ERR_UNSUPPORTED
+
+
+def test_threshold_entry_points_validate_on_the_host(lib):
+    N = None
+    fake = ctypes.c_void_p(1 << 20)
+    d = ctypes.c_double
+    rt = lib.heta_route_threshold
+    rt.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, d] + [ctypes.c_void_p] * 7
+    assert rt(fake, 0, 10, d(0.9), fake, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    assert rt(fake, 1, 0, d(0.9), fake, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    assert rt(fake, 1, 60000, d(0.9), fake, fake, fake, N, N, N, N) == \
+        heta.HETA_ERR_UNSUPPORTED
+    assert rt(fake, 1, 10, d(float("nan")), fake, fake, fake, N, N, N, N) == \
+        heta.HETA_ERR_INVALID_ARG
+    assert rt(fake, 1, 10, d(float("inf")), fake, fake, fake, N, N, N, N) == \
+        heta.HETA_ERR_INVALID_ARG
+    assert rt(fake, 1, 10, d(0.9), N, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert rt(fake, 1, 10, d(0.9), odd, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
+    ac = lib.heta_attention_counts
+    args = [fake, fake, fake, 1, 2, 128, 4, 8, 8, 3, 3, 3, ctypes.c_float(0.1), fake, 256, fake,
+            fake, fake, 1 << 30, N, N]
+    no_counts = list(args)
+    no_counts[15] = N
+    assert ac(*no_counts) == heta.HETA_ERR_INVALID_ARG
+    big_cap = list(args)
+    big_cap[14] = 257
+    assert ac(*big_cap) == heta.HETA_ERR_INVALID_ARG
+    bad_d = list(args)
+    bad_d[5] = 96
+    assert ac(*bad_d) == heta.HETA_ERR_UNSUPPORTED
+    small_ws = list(args)
+    small_ws[18] = 16
+    assert ac(*small_ws) == heta.HETA_ERR_INVALID_ARG
 
 
 def test_flop_model_matches_the_papers_reduction():

@@ -66,6 +66,11 @@ def load():
     lib.heta_attention.restype = i
     lib.heta_uncertainty.argtypes = [vp, vp, f, i, i, i, vp, vp, vp]
     lib.heta_uncertainty.restype = i
+    lib.heta_route_threshold.argtypes = [vp, i, i, d, vp, vp, vp, vp, vp, vp, vp]
+    lib.heta_route_threshold.restype = i
+    lib.heta_attention_counts.argtypes = ([vp, vp, vp] + [i] * 9 +
+                                          [f, vp, i, vp, vp, vp, ctypes.c_size_t, vp, vp])
+    lib.heta_attention_counts.restype = i
     _lib = lib
     return lib
 
@@ -135,6 +140,33 @@ def route(u, k: int, *, out=None, want_thresh=False, want_mask=False, status=Non
     return dense, local, thresh, mask
 
 
+def route_threshold(u, c: float, *, out=None, want_thresh=False, want_mask=False,
+                    status=None):
+    """Routing by the paper's T = mu + c*sigma rule (``heta_route_threshold``).
+
+    u: [B,N] float32 CUDA.  Returns (counts [B] int32, dense_idx [B,N] int32,
+    local_idx [B,N] int32, thresh [B] float64 or None, mask [B,N] uint8 or
+    None), all on the device; row b of dense_idx holds counts[b] ids.
+    ``out`` may pass preallocated (counts, dense_idx, local_idx, thresh, mask).
+    """
+    import torch
+    pu = _dev(u, torch.float32, "u", 2)
+    B, N = u.shape
+    if out is None:
+        counts = torch.empty(B, dtype=torch.int32, device=u.device)
+        dense = torch.empty((B, N), dtype=torch.int32, device=u.device)
+        local = torch.empty((B, N), dtype=torch.int32, device=u.device)
+        thresh = torch.empty(B, dtype=torch.float64, device=u.device) if want_thresh else None
+        mask = torch.empty((B, N), dtype=torch.uint8, device=u.device) if want_mask else None
+    else:
+        counts, dense, local, thresh, mask = out
+    rc = load().heta_route_threshold(pu, B, N, float(c), _opt(counts), _opt(dense),
+                                     _opt(local), _opt(thresh), _opt(mask), _opt(status),
+                                     _stream())
+    _check(rc, "heta_route_threshold")
+    return counts, dense, local, thresh, mask
+
+
 def attention_workspace_size(B, H, d, grid, win, k) -> int:
     """Bytes of device scratch one ``attention`` call needs for these sizes."""
     n = ctypes.c_size_t(0)
@@ -181,6 +213,43 @@ def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=Non
                                float(scale), pd if k > 0 else None, k, po, pw,
                                workspace.numel(), _opt(status), _stream())
     _check(rc, "heta_attention")
+    return out
+
+
+def attention_counts(Q, K, V, grid, win, dense_idx, counts, *, scale=None, out=None,
+                     status=None, workspace=None):
+    """``attention`` with per-sample dense counts on the device
+    (``heta_attention_counts``): dense_idx [B,k_cap] int32 whose row b holds
+    counts[b] increasing ids (e.g. the ``route_threshold`` output, k_cap = N),
+    counts [B] int32 CUDA.  Returns out [B,H,N,d] bfloat16."""
+    import torch
+    pq = _dev(Q, torch.bfloat16, "Q", 4)
+    pk = _dev(K, torch.bfloat16, "K", 4)
+    pv = _dev(V, torch.bfloat16, "V", 4)
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V shapes differ")
+    B, H, N, d = Q.shape
+    Tg, Hg, Wg = grid
+    if Tg * Hg * Wg != N:
+        raise ValueError("grid %s does not hold N=%d tokens" % (grid, N))
+    pd = _dev(dense_idx, torch.int32, "dense_idx", 2)
+    pc = _dev(counts, torch.int32, "counts", 1)
+    if dense_idx.shape[0] != B or counts.shape[0] != B:
+        raise ValueError("dense_idx / counts batch mismatch")
+    k_cap = dense_idx.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    po = _dev(out, torch.bfloat16, "out", 4)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attention_workspace_size(B, H, d, grid, win, k_cap)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=Q.device)
+    pw = _dev(workspace, torch.uint8, "workspace", 1)
+    rc = load().heta_attention_counts(pq, pk, pv, B, H, d, Tg, Hg, Wg, win[0], win[1], win[2],
+                                      float(scale), pd if k_cap > 0 else None, k_cap, pc, po, pw,
+                                      workspace.numel(), _opt(status), _stream())
+    _check(rc, "heta_attention_counts")
     return out
 
 

@@ -63,7 +63,8 @@ constexpr uint32_t kItemConsumers = 1 + 256 + 32;
 struct Params {
     const uint16_t *Q;
     uint16_t *out;
-    const int32_t *dense_idx;
+    const int32_t *dense_idx;  // [B][k]
+    const int32_t *k_dev;      // [B] dense rows per sample (<= k), or null: all k
     int32_t *status;
     int B, H, N, k;
     int Tg, Hg, Wg, wt, wh, ww;
@@ -150,6 +151,7 @@ struct Item {
     int kv_lo, n;    // K/V tiles [kv_lo, kv_lo + n)
     int split;       // DENSE: which key range
     int pair_id;     // DENSE: global pair index (for the split merge)
+    int kb;          // dense rows of sample b (n == 0: a DENSE pair past them, skipped)
 };
 
 __device__ __forceinline__ Item decode(const Params &p, int id)
@@ -180,6 +182,8 @@ __device__ __forceinline__ Item decode(const Params &p, int id)
         it.n = p.n_kv_l;
     }
     it.b = it.bh / p.H;
+    it.kb = p.k_dev ? min(max(__ldg(p.k_dev + it.b), 0), p.k) : p.k;
+    if (it.mode == DENSE && it.tile[0] * kTileRows >= it.kb) it.n = 0;
     return it;
 }
 
@@ -424,6 +428,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 }
                 if (id < 0) break;
                 const Item it = decode(p, id);
+                if (it.n == 0) {  // a DENSE pair past the sample's dense rows: every role skips it
+                    id = next;
+                    continue;
+                }
                 Box bx[2];
                 if (it.mode == LOCAL) {
                     bx[0] = local_box(p, it.tile[0]);
@@ -531,6 +539,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 if (!ok || id < 0) break;
                 const Item it = decode(p, id);
                 const int n = it.n;
+                if (n == 0) continue;
                 const bool dense = it.mode == DENSE;
                 for (int t = 0; t < 2 && ok; ++t)
                     if (!wait(sh.q_full[t], items & 1u)) ok = false;
@@ -620,7 +629,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             __syncwarp();
             const int32_t *dl = p.dense_idx + (int64_t)it.b * p.k;
             const int HW = p.Hg * p.Wg;
-            for (int t = 0; t < 2 && p.k > 0; ++t) {
+            for (int t = 0; t < 2 && it.kb > 0; ++t) {
                 const Box x = local_box(p, it.tile[t]);
                 if (!x.active) continue;
                 const int lo_tok = (x.t0 * p.Hg + x.h0) * p.Wg + x.w0;
@@ -628,7 +637,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                                    (min(x.h0 + kBoxH, p.Hg) - 1) * p.Wg +
                                    min(x.w0 + kBoxW, p.Wg) - 1;
                 // first position with dense_idx >= lo_tok (32-ary search)
-                int lo = 0, hi = p.k;
+                int lo = 0, hi = it.kb;
                 while (hi - lo > 32) {
                     const int step = (hi - lo + 31) / 32;
                     const int pos = lo + lane * step;
@@ -646,7 +655,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 }
                 for (int base = lo;; base += 32) {
                     const int pos = base + lane;
-                    const int v = pos < p.k ? __ldg(dl + pos) : INT32_MAX;
+                    const int v = pos < it.kb ? __ldg(dl + pos) : INT32_MAX;
                     if (v <= hi_tok) {
                         const int tt = v / HW - x.t0, hh = (v / p.Wg) % p.Hg - x.h0,
                                   ww = v % p.Wg - x.w0;
@@ -679,6 +688,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             const int id = pop_item(qi++, ok);
             if (!ok || id < 0) break;
             const Item it = decode(p, id);
+            if (it.n == 0) continue;
             const bool dense = it.mode == DENSE;
             const int tile = it.tile[t];
             const int64_t row0 = (int64_t)it.bh * p.N;
@@ -689,7 +699,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             Box bx;
             if (dense) {
                 const int q = tile * kTileRows + r;
-                row_valid = tile < p.tiles_d && q < p.k;
+                row_valid = tile < p.tiles_d && q < it.kb;
                 if (row_valid) token = __ldg(p.dense_idx + (int64_t)it.b * p.k + q);
                 const uint4 *src = reinterpret_cast<const uint4 *>(p.Q + (row0 + token) * D);
 #pragma unroll
@@ -925,7 +935,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 }  // namespace
 
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
-                        int wh, int ww)
+                        int wh, int ww, bool per_sample_counts)
 {
     AttnPlan pl;
     pl.n_kv_d = (N + kTileKeys - 1) / kTileKeys;
@@ -946,7 +956,7 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     pl.nkh = (min(kBoxH + wh - 1, Hg) + kKvH - 1) / kKvH;
     pl.nkw = (min(kBoxW + ww - 1, Wg) + kKvW - 1) / kKvW;
     pl.n_kv_l = pl.nkt * pl.nkh * pl.nkw;
-    pl.n_local_items = k < N ? B * H * pl.pairs_l : 0;
+    pl.n_local_items = (k < N || per_sample_counts) ? B * H * pl.pairs_l : 0;
     pl.total_items = pl.n_dense_items + pl.n_local_items;
     // workspace: counter | split arrivals | (m,l) partials | O partials
     pl.off_fix = 256;
@@ -966,6 +976,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     p.Q = a.Q;
     p.out = a.out;
     p.dense_idx = a.dense_idx;
+    p.k_dev = a.k_dev;
     p.status = a.status;
     p.B = a.B; p.H = a.H; p.N = a.N; p.k = a.k;
     p.Tg = a.Tg; p.Hg = a.Hg; p.Wg = a.Wg; p.wt = a.wt; p.wh = a.wh; p.ww = a.ww;

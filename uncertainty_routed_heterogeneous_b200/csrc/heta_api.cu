@@ -2,6 +2,8 @@
 // host-side argument checks, then one asynchronous launch sequence each.
 #include <math.h>
 
+#include <cmath>
+
 #include "heta_internal.cuh"
 
 namespace {
@@ -57,6 +59,22 @@ heta_status heta_route(const float *u, int B, int N, int k, int32_t *dense_idx,
                                         static_cast<cudaStream_t>(stream)));
 }
 
+heta_status heta_route_threshold(const float *u, int B, int N, double c, int32_t *counts,
+                                 int32_t *dense_idx, int32_t *local_idx, double *thresh_out,
+                                 uint8_t *mask_out, int32_t *status_dev, void *stream)
+{
+    if (B < 1 || N < 1 || !std::isfinite(c)) return HETA_ERR_INVALID_ARG;
+    if ((int64_t)B * N >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
+    if (N > heta::kRouteMaxN) return HETA_ERR_UNSUPPORTED;
+    if (!u || !counts || !dense_idx || !local_idx) return HETA_ERR_INVALID_ARG;
+    if (!aligned16(u) || !aligned16(counts) || !aligned16(dense_idx) || !aligned16(local_idx) ||
+        (thresh_out && !aligned16(thresh_out)) || (mask_out && !aligned16(mask_out)))
+        return HETA_ERR_INVALID_ARG;
+    return from_cuda(heta::launch_route_threshold(u, B, N, c, counts, dense_idx, local_idx,
+                                                  thresh_out, mask_out, status_dev,
+                                                  static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 
 namespace {
@@ -110,7 +128,35 @@ heta_status heta_attention(const uint16_t *Q, const uint16_t *K, const uint16_t 
     if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
     heta::AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
+    a.k_dev = nullptr;
     a.B = B; a.H = H; a.d = d; a.N = N; a.k = k;
+    a.Tg = Tg; a.Hg = Hg; a.Wg = Wg; a.wt = wt; a.wh = wh; a.ww = ww;
+    a.scale = scale;
+    return from_cuda(heta::launch_attention(a, plan, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                                  int B, int H, int d, int Tg, int Hg, int Wg, int wt, int wh,
+                                  int ww, float scale, const int32_t *dense_idx, int k_cap,
+                                  const int32_t *counts, uint16_t *out, void *workspace,
+                                  size_t workspace_bytes, int32_t *status_dev, void *stream)
+{
+    const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k_cap);
+    if (st != HETA_OK) return st;
+    const int N = Tg * Hg * Wg;
+    if (!(scale > 0.f) || !isfinite(scale)) return HETA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !out || !counts || (k_cap > 0 && !dense_idx) || !workspace)
+        return HETA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
+        !aligned16(counts) || (dense_idx && !aligned16(dense_idx)) || !aligned16(workspace))
+        return HETA_ERR_INVALID_ARG;
+    const heta::AttnPlan plan =
+        heta::plan_attention(B, H, d, N, k_cap, Tg, Hg, Wg, wt, wh, ww, true);
+    if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
+    heta::AttnArgs a;
+    a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
+    a.k_dev = counts;
+    a.B = B; a.H = H; a.d = d; a.N = N; a.k = k_cap;
     a.Tg = Tg; a.Hg = Hg; a.Wg = Wg; a.wt = wt; a.wh = wh; a.ww = ww;
     a.scale = scale;
     return from_cuda(heta::launch_attention(a, plan, workspace, static_cast<cudaStream_t>(stream)));

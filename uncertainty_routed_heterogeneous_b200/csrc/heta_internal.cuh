@@ -22,13 +22,18 @@ cudaError_t launch_route(const float *u, int B, int N, int k, int32_t *dense_idx
                          int32_t *local_idx, float *thresh, uint8_t *mask,
                          int32_t *status, cudaStream_t s);
 
+cudaError_t launch_route_threshold(const float *u, int B, int N, double c, int32_t *counts,
+                                   int32_t *dense_idx, int32_t *local_idx, double *thresh,
+                                   uint8_t *mask, int32_t *status, cudaStream_t s);
+
 cudaError_t launch_uncertainty(const uint16_t *X, const float *w, float bias,
                                int B, int N, int C, float *u, cudaStream_t s);
 
 struct AttnArgs {
     const uint16_t *Q, *K, *V;
     uint16_t *out;
-    const int32_t *dense_idx;
+    const int32_t *dense_idx;  // [B][k] (row stride k)
+    const int32_t *k_dev;      // [B] per-sample dense counts (<= k), or null: all k
     int32_t *status;
     int B, H, d, N, k;
     int Tg, Hg, Wg, wt, wh, ww;
@@ -47,8 +52,10 @@ struct AttnPlan {
 // on it, never the result; the launch itself uses the device's real count.
 constexpr int kPlanSMs = 148;
 
+// k is the dense rows per sample, or their capacity when per_sample_counts
+// (the counts are then only known on the device: LOCAL items are always planned).
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
-                        int wh, int ww);
+                        int wh, int ww, bool per_sample_counts = false);
 
 cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &plan, void *workspace,
                              cudaStream_t s);
