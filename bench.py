@@ -55,6 +55,8 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-window-sweep", action="store_true",
                    help="skip timing the 9^3 / 11^3 / 13^3 windows of the paper's ablation")
+    p.add_argument("--no-threshold-mode", action="store_true",
+                   help="skip timing the paper's mu + c*sigma routing (c = 0.9)")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="minimum host time the cpu_baseline oracle sample runs for")
     return p.parse_args()
@@ -386,6 +388,44 @@ def run_heta(args, info):
                 "speedup_vs_dense": (dense_cmp["ms"] / ms_n) if dense_cmp else None}
         del ws_n
 
+    # ---- the paper's own threshold rule, T = mu + c*sigma (Eq. (11)), c = 0.9 --
+    thr = None
+    if not args.no_threshold_mode:
+        c = 0.9
+        t_counts = torch.empty(w.B, dtype=torch.int32, device=dev)
+        t_dense = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
+        t_local = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
+        ws_t = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, w.N),
+                           dtype=torch.uint8, device=dev)
+
+        def thr_step(ev=None):
+            if ev is not None:
+                ev[0].record()
+            heta.route_threshold(d_u, c, out=(t_counts, t_dense, t_local, None, None))
+            if ev is not None:
+                ev[1].record()
+            heta.attention_counts(d_Q, d_K, d_V, w.grid, w.win, t_dense, t_counts, out=out,
+                                  workspace=ws_t)
+            if ev is not None:
+                ev[2].record()
+
+        for _ in range(3):
+            thr_step()
+        torch.cuda.synchronize()
+        tev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(10)]
+        for ev in tev:
+            thr_step(ev)
+        torch.cuda.synchronize()
+        cnt = t_counts.cpu().tolist()
+        r_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in tev)
+        a_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in tev)
+        fl_t = sum(heta.attention_flops(1, w.H, w.d, w.N, kb, w.M) for kb in cnt)
+        thr = {"c": c, "dense_counts": cnt, "dense_fraction": sum(cnt) / (w.B * w.N),
+               "route_ms": r_ms, "attention_ms": a_ms,
+               "algorithmic_tflops": fl_t / (a_ms * 1e9),
+               "tokens_per_s": w.B * w.N / ((r_ms + a_ms) / 1e3)}
+        del ws_t
+
     # ---- end to end through the public API with host buffers ----------------
     e2e = None
     if not args.no_e2e:
@@ -446,6 +486,7 @@ def run_heta(args, info):
                           "peak": peaks["hbm_gbs"], "unit": "GB/s"},
         "dense_compare": dense_cmp,
         "window_sweep": win_sweep,
+        "threshold_mode": thr,
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu, "clocks": sampler.summary(),
     }

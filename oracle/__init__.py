@@ -98,7 +98,7 @@ def route(u: np.ndarray, k: int):
 
 
 def route_threshold(u: np.ndarray, c: float):
-    """Routing by the paper's threshold T = mu + c*sigma (Eq. (11)-(12), reading R8).
+    """Routing by the paper's threshold T = mu + c*sigma (Eq. (11)-(12), reading R10).
 
     u: [B,N] float32.  Returns (counts [B], dense_idx [B,N], local_idx [B,N],
     thresh [B] float64, mask [B,N]); row b of dense_idx holds counts[b]

@@ -36,7 +36,7 @@
  *   R7 the uncertainty head is u = softplus(x . w + b).  The paper names it
  *      only as a "lightweight branch" with u >= 0; a linear map followed by
  *      softplus is the plainest form that satisfies Eq. (7).
- *   R8 threshold mode (the paper's own rule): mu and sigma are the mean and
+ *   R10 threshold mode (the paper's own rule): mu and sigma are the mean and
  *      the population standard deviation of one sample's N uncertainties,
  *      in fp64; u == T goes dense (Eq. (12)'s strict "<").  The count then
  *      varies per sample.
@@ -117,7 +117,7 @@ int oracle_route(const float *u, int B, int N, int k,
 }
 
 /* ------------------------------------------------------------------ */
-/* Routing by the paper's own threshold rule, Eq. (11)-(12) (R8).      */
+/* Routing by the paper's own threshold rule, Eq. (11)-(12) (R10).     */
 /* ------------------------------------------------------------------ */
 
 /*

@@ -251,7 +251,7 @@ def test_route_nan_is_an_error():
 
 
 # --------------------------------------------------------------------------
-# threshold routing, the paper's own rule (Eq. (11)-(12), reading R8)
+# threshold routing, the paper's own rule (Eq. (11)-(12), reading R10)
 # --------------------------------------------------------------------------
 
 def read_threshold_golden():
