@@ -57,6 +57,8 @@ def parse_args():
                    help="skip timing the 9^3 / 11^3 / 13^3 windows of the paper's ablation")
     p.add_argument("--no-threshold-mode", action="store_true",
                    help="skip timing the paper's mu + c*sigma routing (c = 0.9)")
+    p.add_argument("--no-route-throughput", action="store_true",
+                   help="skip timing heta_route on 512 samples in one launch")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="minimum host time the cpu_baseline oracle sample runs for")
     return p.parse_args()
@@ -426,6 +428,34 @@ def run_heta(args, info):
                "tokens_per_s": w.B * w.N / ((r_ms + a_ms) / 1e3)}
         del ws_t
 
+    # ---- routing in throughput mode: 512 samples of this N in one launch -------
+    route_tp = None
+    if not args.no_route_throughput:
+        Bt = 512
+        g = torch.Generator(device=dev)
+        g.manual_seed(7)
+        u_tp = (d_u[:1].repeat(Bt, 1) +
+                1e-3 * torch.randn((Bt, w.N), generator=g, device=dev)).contiguous()
+        dn_tp = torch.empty((Bt, kk), dtype=torch.int32, device=dev)
+        lc_tp = torch.empty((Bt, w.N - kk), dtype=torch.int32, device=dev)
+        for _ in range(3):
+            heta.route(u_tp, kk, out=(dn_tp, lc_tp, None, None))
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        e0.record()
+        for _ in range(reps):
+            heta.route(u_tp, kk, out=(dn_tp, lc_tp, None, None))
+        e1.record()
+        torch.cuda.synchronize()
+        us = 1e3 * e0.elapsed_time(e1) / reps
+        nbytes = Bt * w.N * 4 * 2  # read u once, write both index lists
+        hbm = load_peaks()["hbm_gbs"]
+        route_tp = {"B": Bt, "N": w.N, "k": kk, "us": us, "bytes": nbytes,
+                    "GB/s": nbytes / (us * 1e3), "frac_of_hbm": nbytes / (us * 1e3) / hbm,
+                    "peak_source": "measured copy bandwidth"}
+        del u_tp, dn_tp, lc_tp
+
     # ---- end to end through the public API with host buffers ----------------
     e2e = None
     if not args.no_e2e:
@@ -487,6 +517,7 @@ def run_heta(args, info):
         "dense_compare": dense_cmp,
         "window_sweep": win_sweep,
         "threshold_mode": thr,
+        "route_throughput": route_tp,
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu, "clocks": sampler.summary(),
     }

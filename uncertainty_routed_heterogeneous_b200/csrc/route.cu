@@ -6,10 +6,13 @@
 // equal u are taken in increasing token index; -0.0 == +0.0.
 //
 // One CTA per sample.  The sample's u is read from HBM once (coalesced
-// 16-byte loads) into shared memory as order-preserving uint32 keys; four
-// 8-bit radix passes in shared memory find the k-th largest key K* and how
-// many keys equal to K* are taken; a last pass compacts both index lists in
-// increasing order with warp ballots and writes them as contiguous runs.
+// 16-byte loads) into shared memory as order-preserving uint32 keys, and the
+// histogram of their top 11 bits is counted on the way in; two more radix
+// passes over the keys (the next 11 bits, the last 10) count only the keys
+// still in the running, so after the first pass almost every key costs a
+// compare.  That finds the k-th largest key K* and how many keys equal to K*
+// are taken; a last pass compacts both index lists in increasing order with
+// warp ballots and writes them as contiguous runs.
 #include "heta_internal.cuh"
 
 namespace heta {
@@ -33,6 +36,53 @@ __device__ __forceinline__ float key_value(uint32_t key)
     return __uint_as_float(b);
 }
 
+// The digit of the r-th largest key among those counted in hist[0..nbins)
+// (nbins = 1024 or 2048): *digit and *rank_in_digit (1-based) for the next
+// pass.  Bins are scanned from the top; every thread of the CTA calls this.
+__device__ __forceinline__ void find_digit(const uint32_t *hist, int nbins, uint32_t r,
+                                           uint32_t *warp_tot, uint32_t *s_digit,
+                                           uint32_t *s_rank)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int per = nbins / kThreads;  // 1 or 2 bins per thread, descending
+    uint32_t c[2] = {0u, 0u}, sum = 0u;
+    for (int j = 0; j < per; ++j) {
+        c[j] = hist[nbins - 1 - per * tid - j];
+        sum += c[j];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    uint32_t wbefore = 0u;
+    {
+        const uint32_t wt = warp_tot[lane];
+        uint32_t wi = wt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += t;
+        }
+        wbefore = __shfl_sync(0xffffffffu, wi - wt, warp);
+    }
+    const uint32_t before = wbefore + incl - sum;
+    if (before < r && r <= before + sum) {
+        uint32_t acc = before;
+        for (int j = 0; j < per; ++j) {
+            if (acc < r && r <= acc + c[j]) {
+                *s_digit = (uint32_t)(nbins - 1 - per * tid - j);
+                *s_rank = r - acc;
+            }
+            acc += c[j];
+        }
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 route_kernel(const float *__restrict__ u, int N, int k,
              int32_t *__restrict__ dense_idx, int32_t *__restrict__ local_idx,
@@ -40,8 +90,9 @@ route_kernel(const float *__restrict__ u, int N, int k,
              int32_t *status)
 {
     extern __shared__ uint32_t keys[];
-    __shared__ uint32_t hist[256];
-    __shared__ uint32_t s_prefix, s_take;
+    __shared__ uint32_t hist[2048];
+    __shared__ uint32_t warp_tot[kWarps];
+    __shared__ uint32_t s_digit, s_rank;
     __shared__ uint32_t w_gt[kWarps], w_eq[kWarps];
     __shared__ uint32_t w_dense_before[kWarps], w_eq_before[kWarps];
     __shared__ int s_nan;
@@ -50,111 +101,115 @@ route_kernel(const float *__restrict__ u, int N, int k,
     const int b = blockIdx.x;
     const float *ub = u + (size_t)b * N;
     if (tid == 0) s_nan = 0;
+    for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
     __syncthreads();
 
-    // ---- 1. one coalesced read of u into shared memory as keys ----------
+    // ---- 1. one coalesced read of u into shared memory as keys, counting
+    // the histogram of their top 11 bits on the way
     bool nan_seen = false;
+    auto put = [&](int i, float f) {
+        nan_seen |= (f != f);
+        const uint32_t key = order_key(f);
+        keys[i] = key;
+        atomicAdd(&hist[key >> 21], 1u);
+    };
     int head = 0;  // scalar elements before the first 16-byte boundary
     {
         uintptr_t a = reinterpret_cast<uintptr_t>(ub);
         head = (int)(((16u - (a & 15u)) & 15u) >> 2);
         if (head > N) head = N;
     }
-    if (tid < head) {
-        float f = __ldg(ub + tid);
-        nan_seen |= (f != f);
-        keys[tid] = order_key(f);
-    }
+    if (tid < head) put(tid, __ldg(ub + tid));
     const int n4 = (N - head) >> 2;
     const float4 *u4 = reinterpret_cast<const float4 *>(ub + head);
-    for (int v = tid; v < n4; v += kThreads) {
-        float4 f = __ldg(u4 + v);
-        nan_seen |= (f.x != f.x) | (f.y != f.y) | (f.z != f.z) | (f.w != f.w);
-        int i = head + 4 * v;
-        keys[i] = order_key(f.x);
-        keys[i + 1] = order_key(f.y);
-        keys[i + 2] = order_key(f.z);
-        keys[i + 3] = order_key(f.w);
+    // four loads in flight per thread before their keys are stored
+    for (int v0 = tid; v0 < n4; v0 += 4 * kThreads) {
+        float4 f[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int v = v0 + q * kThreads;
+            f[q] = v < n4 ? __ldg(u4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int v = v0 + q * kThreads;
+            if (v < n4) {
+                const int i = head + 4 * v;
+                put(i, f[q].x);
+                put(i + 1, f[q].y);
+                put(i + 2, f[q].z);
+                put(i + 3, f[q].w);
+            }
+        }
     }
-    for (int i = head + 4 * n4 + tid; i < N; i += kThreads) {
-        float f = __ldg(ub + i);
-        nan_seen |= (f != f);
-        keys[i] = order_key(f);
-    }
+    for (int i = head + 4 * n4 + tid; i < N; i += kThreads) put(i, __ldg(ub + i));
     if (nan_seen) s_nan = 1;
     __syncthreads();
     if (tid == 0 && s_nan) raise_status(status, HETA_ERR_NONFINITE);
 
-    // ---- 2. radix select of the k-th largest key --------------------------
+    // ---- 2. radix select of the k-th largest key: digits of 11, 11, 10 bits
     uint32_t kstar = 0xffffffffu, take = 0u;  // k == 0: nothing is dense
     if (k > 0) {
-        uint32_t prefix = 0u, remaining = (uint32_t)k;
-        const int iters = (N + kThreads - 1) / kThreads;
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            const uint32_t hi_mask = pass == 0 ? 0u : (0xffffffffu << (shift + 8));
-            if (tid < 256) hist[tid] = 0u;
-            __syncthreads();
-            for (int it = 0; it < iters; ++it) {
-                const int i = it * kThreads + tid;
-                uint32_t digit = 256u;  // sentinel: not counted
-                if (i < N) {
-                    uint32_t key = keys[i];
-                    if ((key & hi_mask) == prefix) digit = (key >> shift) & 255u;
-                }
-                // lanes holding the same digit add once, through their leader
-                unsigned peers = __match_any_sync(0xffffffffu, digit);
-                if (digit < 256u && lane == __ffs(peers) - 1)
-                    atomicAdd(&hist[digit], (uint32_t)__popc(peers));
-            }
-            __syncthreads();
-            if (warp == 0) {
-                // lane l holds bins 255-8l .. 248-8l (descending)
-                uint32_t c[8], sum = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    c[j] = hist[255 - 8 * lane - j];
-                    sum += c[j];
-                }
-                uint32_t incl = sum;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += t;
-                }
-                const uint32_t before = incl - sum;
-                if (before < remaining && remaining <= incl) {
-                    uint32_t acc = before;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        if (acc < remaining && remaining <= acc + c[j]) {
-                            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
-                            s_take = remaining - acc;
-                        }
-                        acc += c[j];
-                    }
-                }
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            remaining = s_take;
+        find_digit(hist, 2048, (uint32_t)k, warp_tot, &s_digit, &s_rank);
+        const uint32_t d1 = s_digit, r1 = s_rank;
+        for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
+        __syncthreads();
+        const uint4 *keys4 = reinterpret_cast<const uint4 *>(keys);
+        for (int v = tid; v < (N >> 2); v += kThreads) {
+            const uint4 q = keys4[v];
+            if ((q.x >> 21) == d1) atomicAdd(&hist[(q.x >> 10) & 2047u], 1u);
+            if ((q.y >> 21) == d1) atomicAdd(&hist[(q.y >> 10) & 2047u], 1u);
+            if ((q.z >> 21) == d1) atomicAdd(&hist[(q.z >> 10) & 2047u], 1u);
+            if ((q.w >> 21) == d1) atomicAdd(&hist[(q.w >> 10) & 2047u], 1u);
         }
-        kstar = prefix;
-        take = remaining;
+        for (int i = 4 * (N >> 2) + tid; i < N; i += kThreads) {
+            const uint32_t key = keys[i];
+            if ((key >> 21) == d1) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
+        }
+        __syncthreads();
+        find_digit(hist, 2048, r1, warp_tot, &s_digit, &s_rank);
+        const uint32_t p2 = (d1 << 11) | s_digit, r2 = s_rank;
+        for (int i = tid; i < 1024; i += kThreads) hist[i] = 0u;
+        __syncthreads();
+        for (int v = tid; v < (N >> 2); v += kThreads) {
+            const uint4 q = keys4[v];
+            if ((q.x >> 10) == p2) atomicAdd(&hist[q.x & 1023u], 1u);
+            if ((q.y >> 10) == p2) atomicAdd(&hist[q.y & 1023u], 1u);
+            if ((q.z >> 10) == p2) atomicAdd(&hist[q.z & 1023u], 1u);
+            if ((q.w >> 10) == p2) atomicAdd(&hist[q.w & 1023u], 1u);
+        }
+        for (int i = 4 * (N >> 2) + tid; i < N; i += kThreads) {
+            const uint32_t key = keys[i];
+            if ((key >> 10) == p2) atomicAdd(&hist[key & 1023u], 1u);
+        }
+        __syncthreads();
+        find_digit(hist, 1024, r2, warp_tot, &s_digit, &s_rank);
+        kstar = (p2 << 10) | s_digit;
+        take = s_rank;
     }
     if (tid == 0 && thresh)
         thresh[b] = k > 0 ? key_value(kstar) : __uint_as_float(0x7f800000u);
 
     // ---- 3. compaction: each warp owns one contiguous segment -------------
-    const int per_lane = (N + kThreads - 1) / kThreads;
+    // (segments hold a multiple of 128 keys, so the counts read 16 bytes a lane)
+    const int per_lane = ((N + kThreads - 1) / kThreads + 3) & ~3;
     const int seg = 32 * per_lane;
-    const int seg_lo = warp * seg;
+    const int seg_lo = min(N, warp * seg);
     const int seg_hi = min(N, seg_lo + seg);
     uint32_t n_gt = 0, n_eq = 0;
-    for (int i = seg_lo + lane; i < seg_hi; i += 32) {
-        uint32_t key = keys[i];
-        n_gt += key > kstar;
-        n_eq += key == kstar;
+    {
+        const int full4 = (seg_hi - seg_lo) >> 2;  // whole uint4 of the segment
+        const uint4 *k4 = reinterpret_cast<const uint4 *>(keys + seg_lo);
+        for (int v = lane; v < full4; v += 32) {
+            const uint4 q = k4[v];
+            n_gt += (q.x > kstar) + (q.y > kstar) + (q.z > kstar) + (q.w > kstar);
+            n_eq += (q.x == kstar) + (q.y == kstar) + (q.z == kstar) + (q.w == kstar);
+        }
+        for (int i = seg_lo + 4 * full4 + lane; i < seg_hi; i += 32) {
+            const uint32_t key = keys[i];
+            n_gt += key > kstar;
+            n_eq += key == kstar;
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
