@@ -42,6 +42,10 @@ def _load():
                                      ctypes.c_void_p]
         lib.oracle_route_threshold.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_double] + [ctypes.c_void_p] * 5
+        lib.oracle_philox4x32_10.argtypes = [ctypes.c_void_p] * 3
+        lib.oracle_route_swap.argtypes = ([ctypes.c_void_p] + [ctypes.c_int] * 4 +
+                                          [ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p,
+                                           ctypes.c_void_p])
         lib.oracle_window_start.argtypes = [ctypes.c_int] * 3
         lib.oracle_window.argtypes = [ctypes.c_int] * 7 + [ctypes.c_void_p]
         lib.oracle_attention_rows.argtypes = (
@@ -117,6 +121,31 @@ def route_threshold(u: np.ndarray, c: float):
     if rc:
         raise OracleError(rc)
     return counts, dense, local, thresh, mask
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 (Salmon et al., SC 2011) of a 4-word counter and 2-word key."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.zeros(4, np.uint32)
+    _load().oracle_philox4x32_10(_ptr(c), _ptr(k), _ptr(out))
+    return out
+
+
+def route_swap(dense_idx: np.ndarray, N: int, s: int, seed: int, block: int):
+    """One transformer block's random swap (reading R11) of a top-k routing.
+
+    dense_idx: [B,k] int32 ascending.  Returns (dense [B,k], local [B,N-k]).
+    """
+    dense_idx = np.ascontiguousarray(dense_idx, dtype=np.int32)
+    B, k = dense_idx.shape
+    dense = np.zeros((B, k), np.int32)
+    local = np.zeros((B, N - k), np.int32)
+    rc = _load().oracle_route_swap(_ptr(dense_idx), B, int(N), int(k), int(s), int(seed),
+                                   int(block), _ptr(dense), _ptr(local))
+    if rc:
+        raise OracleError(rc)
+    return dense, local
 
 
 def window_start(p: int, extent: int, width: int) -> int:

@@ -40,6 +40,15 @@
  *      the population standard deviation of one sample's N uncertainties,
  *      in fp64; u == T goes dense (Eq. (12)'s strict "<").  The count then
  *      varies per sample.
+ *   R11 per-block random swap: at transformer block `block`, s tokens of
+ *      the dense set (a uniformly random subset) trade places with s
+ *      uniformly random tokens of the local set, so the count stays k.
+ *      The swap ratio r of Table 8 is read as a fraction of N (s = ceil(rN),
+ *      decimal-snapped as for k), which makes r = rho fully random as the
+ *      paper's "fully random selection at 20%" says.  The subsets are the s
+ *      smallest (rho_i, i) of each set, rho_i = Philox4x32-10 word 0 with
+ *      counter (i, b, block, 0) and key (seed low, seed high): any side can
+ *      reproduce them from the seed.
  *
  * All arithmetic is IEEE fp64 on inputs that are exactly representable
  * (fp32 arrays holding bf16 values, or fp32 values), in plain loop order.
@@ -159,6 +168,115 @@ int oracle_route_threshold(const float *u, int B, int N, double c, int32_t *coun
         counts[b] = nd;
     }
     return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-block random swap (§3.2.2 after Eq. (12); App. B Table 8), R11. */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Philox4x32-10, the counter-based generator of Salmon, Moraes, Dror and
+ * Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC 2011): ten rounds
+ * of two 32x32->64 multiplications (multipliers 0xD2511F53, 0xCD9E8D57) whose
+ * halves are mixed with the other counter words and the key; the key is
+ * advanced by the Weyl increments 0x9E3779B9, 0xBB67AE85 before every round
+ * after the first.
+ */
+void oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+        const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+        c0 = hi1 ^ c1 ^ k0;
+        c1 = lo1;
+        c2 = hi0 ^ c3 ^ k1;
+        c3 = lo0;
+    }
+    out[0] = c0;
+    out[1] = c1;
+    out[2] = c2;
+    out[3] = c3;
+}
+
+/* The random draw of token i of sample b at transformer block `block`. */
+static uint32_t swap_draw(int i, int b, int block, uint64_t seed)
+{
+    const uint32_t ctr[4] = {(uint32_t)i, (uint32_t)b, (uint32_t)block, 0u};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    oracle_philox4x32_10(ctr, key, out);
+    return out[0];
+}
+
+static const uint32_t *g_sort_draw; /* qsort has no context pointer */
+
+static int order_draw_then_index(const void *pa, const void *pb)
+{
+    int32_t a = *(const int32_t *)pa, b = *(const int32_t *)pb;
+    if (g_sort_draw[a] < g_sort_draw[b]) return -1;
+    if (g_sort_draw[a] > g_sort_draw[b]) return 1;
+    return (a < b) ? -1 : (a > b) ? 1 : 0;
+}
+
+/*
+ * One block's swap, per sample b: every token i draws rho_i (above); of the
+ * dense set D (dense_idx row b, k entries) the s tokens with the smallest
+ * (rho_i, i) go local, and of its complement the s tokens with the smallest
+ * (rho_i, i) go dense.  Writes the new sets, ascending, to dense_out [B,k]
+ * and local_out [B,N-k].  Requires 0 <= s <= min(k, N-k) and a valid
+ * dense_idx (distinct ids in [0,N)); otherwise status 1.
+ */
+int oracle_route_swap(const int32_t *dense_idx, int B, int N, int k, int s, uint64_t seed,
+                      int block, int32_t *dense_out, int32_t *local_out)
+{
+    if (B < 0 || N < 0 || k < 0 || k > N || s < 0 || s > k || s > N - k)
+        return ORACLE_INVALID;
+    uint8_t *dense = (uint8_t *)malloc((size_t)(N > 0 ? N : 1));
+    uint32_t *draw = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)(N > 0 ? N : 1));
+    int32_t *gd = (int32_t *)malloc(sizeof(int32_t) * (size_t)(k > 0 ? k : 1));
+    int32_t *gl = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N - k > 0 ? N - k : 1));
+    int rc = ORACLE_OK;
+    if (!dense || !draw || !gd || !gl) rc = ORACLE_INVALID;
+    for (int b = 0; b < B && rc == ORACLE_OK; ++b) {
+        memset(dense, 0, (size_t)N);
+        for (int j = 0; j < k; ++j) {
+            const int32_t t = dense_idx[(int64_t)b * k + j];
+            if (t < 0 || t >= N || dense[t]) { rc = ORACLE_INVALID; break; }
+            dense[t] = 1;
+        }
+        if (rc != ORACLE_OK) break;
+        int nd = 0, nl = 0;
+        for (int i = 0; i < N; ++i) {
+            draw[i] = swap_draw(i, b, block, seed);
+            if (dense[i]) gd[nd++] = i;
+            else gl[nl++] = i;
+        }
+        g_sort_draw = draw;
+        qsort(gd, (size_t)nd, sizeof(int32_t), order_draw_then_index);
+        qsort(gl, (size_t)nl, sizeof(int32_t), order_draw_then_index);
+        for (int j = 0; j < s; ++j) {
+            dense[gd[j]] = 0;
+            dense[gl[j]] = 1;
+        }
+        nd = nl = 0;
+        for (int i = 0; i < N; ++i) {
+            if (dense[i]) dense_out[(int64_t)b * k + nd++] = i;
+            else local_out[(int64_t)b * (N - k) + nl++] = i;
+        }
+    }
+    free(dense);
+    free(draw);
+    free(gd);
+    free(gl);
+    return rc;
 }
 
 /* ------------------------------------------------------------------ */

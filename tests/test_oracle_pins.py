@@ -16,6 +16,10 @@ What pins what:
   * threshold    -- hand-worked mu + c*sigma cases (golden/route_threshold.txt),
                     numpy's mean/std (ddof=0) in fp64, the Gaussian tail
                     fraction 1 - Phi(c), shift/scale invariance, u == T dense
+  * swap         -- Philox4x32-10 known-answer vectors (golden/philox_kat.txt),
+                    a brute-force restatement on small inputs (sorting the
+                    draws), set sizes and identities, and the coverage
+                    1 - (1 - s/(N-k))^30 over 30 blocks
   * attention    -- torch's scaled_dot_product_attention in fp64 (a library
                     routine) with no mask (rho = 1) and with a boolean window
                     mask built from the independent window definition (rho=0);
@@ -360,6 +364,93 @@ def test_threshold_edge_cases():
     assert counts.tolist() == [5, 5]
     assert d[0, :5].tolist() == [5, 6, 7, 8, 9] and d[1, :5].tolist() == [0, 1, 2, 3, 4]
     assert thresh.tolist() == [4.5, -4.5]
+
+
+# --------------------------------------------------------------------------
+# per-block random swap (§3.2.2, App. B Table 8; reading R11)
+# --------------------------------------------------------------------------
+
+def read_philox_kat():
+    cases = []
+    for line in open(os.path.join(GOLDEN, "philox_kat.txt")):
+        line = line.split("#")[0].strip()
+        if line:
+            ctr, key, out = ([int(x, 16) for x in f.split()] for f in line.split("|"))
+            cases.append((ctr, key, out))
+    return cases
+
+
+@pytest.mark.parametrize("case", read_philox_kat())
+def test_philox_known_answers(case):
+    ctr, key, out = case
+    assert oracle.philox4x32_10(ctr, key).tolist() == out
+
+
+def _draws_bruteforce(N, b, block, seed):
+    """rho_i for every token, from the oracle's Philox (pinned above)."""
+    return [int(oracle.philox4x32_10([i, b, block, 0],
+                                     [seed & 0xffffffff, seed >> 32])[0]) for i in range(N)]
+
+
+@pytest.mark.parametrize("N,k,s", [(40, 12, 5), (33, 16, 16), (64, 1, 1), (50, 30, 0)])
+def test_swap_vs_bruteforce(N, k, s):
+    rng = np.random.default_rng(N + k)
+    u = rng.random((2, N), dtype=np.float32)
+    dense, _, _ = oracle.route(u, k)
+    seed, block = 0x123456789ABCDEF, 7
+    got_d, got_l = oracle.route_swap(dense, N, s, seed, block)
+    for b in range(2):
+        draw = _draws_bruteforce(N, b, block, seed)
+        D = [int(i) for i in dense[b]]
+        L = [i for i in range(N) if i not in set(D)]
+        out_d = sorted(D, key=lambda i: (draw[i], i))[:s]
+        in_l = sorted(L, key=lambda i: (draw[i], i))[:s]
+        want = sorted((set(D) - set(out_d)) | set(in_l))
+        assert got_d[b].tolist() == want
+        assert got_l[b].tolist() == sorted(set(range(N)) - set(want))
+
+
+def test_swap_identities():
+    rng = np.random.default_rng(1)
+    u = rng.random((3, 500), dtype=np.float32)
+    dense, local, _ = oracle.route(u, 250)
+    d0, l0 = oracle.route_swap(dense, 500, 0, 9, 0)
+    assert np.array_equal(d0, dense) and np.array_equal(l0, local)
+    # s = k = N - k swaps every token
+    d1, l1 = oracle.route_swap(dense, 500, 250, 9, 0)
+    assert np.array_equal(d1, local) and np.array_equal(l1, dense)
+    # s of each: sizes, overlaps, and a different draw per block and per sample
+    d2, _ = oracle.route_swap(dense, 500, 35, 9, 0)
+    d3, _ = oracle.route_swap(dense, 500, 35, 9, 1)
+    for b in range(3):
+        assert len(set(d2[b]) & set(dense[b])) == 250 - 35
+        assert len(set(d2[b]) - set(dense[b])) == 35
+    assert not np.array_equal(d2, d3)
+    assert not np.array_equal(np.setdiff1d(d2[0], dense[0]), np.setdiff1d(d2[1], dense[1]))
+    with pytest.raises(oracle.OracleError):
+        oracle.route_swap(dense, 500, 251, 9, 0)
+
+
+def test_swap_coverage_over_30_blocks():
+    """Table 8's setting: r = 7% of N swapped per block, 30 blocks.  A token
+    outside D is drawn with probability p = s/(N-k) per block, so the share
+    of them dense at least once is 1 - (1-p)^30 (the paper's 1 - (1-r)^30 =
+    0.89 takes p = r); the dense tokens keep their place with probability
+    1 - s/k per block."""
+    N = 32760
+    k = oracle.dense_count(N, 0.2)
+    s = min(oracle.dense_count(N, 0.07), k, N - k)
+    u = W.make_u(W.WAN21)
+    dense, local, _ = oracle.route(u, k)
+    seen = np.zeros(N, bool)
+    kept = []
+    for block in range(30):
+        d, _ = oracle.route_swap(dense, N, s, 2024, block)
+        seen[d[0]] = True
+        kept.append(len(np.intersect1d(d[0], dense[0])) / k)
+    p = s / (N - k)
+    assert abs(seen[local[0]].mean() - (1 - (1 - p) ** 30)) < 0.01
+    assert abs(np.mean(kept) - (1 - s / k)) < 1e-12
 
 
 # --------------------------------------------------------------------------
