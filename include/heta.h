@@ -96,6 +96,36 @@ HETA_API heta_status heta_route(const float *u, int B, int N, int k,
                        int32_t *status_dev, void *stream);
 
 /*
+ * heta_route_swap -- the per-block random swap of a top-k routing (§3.2.2,
+ * after Eq. (12); App. B Table 8): at transformer block `block`, s tokens of
+ * each sample's dense set trade places with s tokens of its local set, so
+ * uncertain tokens keep dense attention most of the time while others get
+ * some.  The tokens are chosen by a counter-based generator any program can
+ * reproduce: token i of sample b draws rho_i = word 0 of Philox4x32-10
+ * (Salmon et al., SC 2011) with counter (i, b, block, 0) and key
+ * (seed & 0xffffffff, seed >> 32); the s dense tokens with the smallest
+ * (rho_i, i) go local and the s local tokens with the smallest (rho_i, i) go
+ * dense.  The paper's swap ratio r (7% by default) gives s = ceil(r*N) (the
+ * heta_dense_count of r), at most min(k, N-k).
+ *
+ *   dense_idx  [B,k] int32: a routing's dense sets, distinct ids in [0,N)
+ *              (the heta_route output).  An id out of range raises status_dev
+ *              to HETA_ERR_INVALID_ARG and that sample's outputs are not
+ *              written; repeated ids give unspecified outputs.
+ *   dense_out  [B,k] int32 out: the new dense sets, increasing.  May be
+ *              dense_idx itself (each sample's row is read before written).
+ *   local_out  [B,N-k] int32 out: the complements, increasing.
+ *   mask_out   [B,N] uint8 out, or NULL: m_i of the new sets, 1 = local.
+ *
+ * Requires 0 <= s <= min(k, N-k), block >= 0 and the heta_route size limits;
+ * pointers 16-byte aligned.  One CTA per sample.
+ */
+HETA_API heta_status heta_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
+                                     uint64_t seed, int block, int32_t *dense_out,
+                                     int32_t *local_out, uint8_t *mask_out,
+                                     int32_t *status_dev, void *stream);
+
+/*
  * heta_route_threshold -- routing by the paper's own rule (Eq. (11)-(12)):
  * per sample b, T_b = mu_b + c * sigma_b, where mu_b and sigma_b are the mean
  * and the population standard deviation of u[b,:], computed in fp64; token i

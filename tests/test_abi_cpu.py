@@ -35,7 +35,7 @@ def test_header_declares_the_three_path_calls():
     names = declared_symbols()
     assert {"heta_route", "heta_attention", "heta_uncertainty", "heta_dense_count",
             "heta_status_string", "heta_version", "heta_attention_workspace_size",
-            "heta_route_threshold", "heta_attention_counts"} <= names
+            "heta_route_threshold", "heta_attention_counts", "heta_route_swap"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -134,6 +134,33 @@ def test_threshold_entry_points_validate_on_the_host(lib):
     small_ws = list(args)
     small_ws[18] = 16
     assert ac(*small_ws) == heta.HETA_ERR_INVALID_ARG
+
+
+def test_swap_entry_point_validates_on_the_host(lib):
+    N = None
+    fake = ctypes.c_void_p(1 << 20)
+    sw = lib.heta_route_swap
+    sw.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_uint64, ctypes.c_int] + \
+        [ctypes.c_void_p] * 5
+    ok = [fake, 1, 100, 20, 5, 7, 0, fake, fake, N, N, N]
+    for pos, bad in ((1, 0), (2, 0), (3, 101), (4, 21), (4, -1), (6, -1)):
+        a = list(ok)
+        a[pos] = bad
+        assert sw(*a) == heta.HETA_ERR_INVALID_ARG, (pos, bad)
+    big_s = list(ok)
+    big_s[3], big_s[4] = 90, 11  # s > N - k
+    assert sw(*big_s) == heta.HETA_ERR_INVALID_ARG
+    too_big = list(ok)
+    too_big[2], too_big[3], too_big[4] = 60000, 20, 5
+    assert sw(*too_big) == heta.HETA_ERR_UNSUPPORTED
+    no_local = list(ok)
+    no_local[8] = N
+    assert sw(*no_local) == heta.HETA_ERR_INVALID_ARG
+    odd = list(ok)
+    odd[7] = ctypes.c_void_p((1 << 20) + 4)
+    assert sw(*odd) == heta.HETA_ERR_INVALID_ARG
+    assert heta.swap_count(32760, 6552, 0.07) == 2294
+    assert heta.swap_count(100, 5, 0.07) == 5
 
 
 def test_flop_model_matches_the_papers_reduction():

@@ -66,6 +66,8 @@ def load():
     lib.heta_attention.restype = i
     lib.heta_uncertainty.argtypes = [vp, vp, f, i, i, i, vp, vp, vp]
     lib.heta_uncertainty.restype = i
+    lib.heta_route_swap.argtypes = [vp, i, i, i, i, ctypes.c_uint64, i, vp, vp, vp, vp, vp]
+    lib.heta_route_swap.restype = i
     lib.heta_route_threshold.argtypes = [vp, i, i, d, vp, vp, vp, vp, vp, vp, vp]
     lib.heta_route_threshold.restype = i
     lib.heta_attention_counts.argtypes = ([vp, vp, vp] + [i] * 9 +
@@ -138,6 +140,38 @@ def route(u, k: int, *, out=None, want_thresh=False, want_mask=False, status=Non
                            _opt(status), _stream())
     _check(rc, "heta_route")
     return dense, local, thresh, mask
+
+
+def swap_count(N: int, k: int, r: float) -> int:
+    """Tokens one block's random swap moves each way: ceil(r*N) (read like
+    ``dense_count``), at most min(k, N-k)."""
+    return min(dense_count(N, r), k, N - k)
+
+
+def route_swap(dense_idx, N: int, s: int, seed: int, block: int, *, out=None, want_mask=False,
+               status=None):
+    """One transformer block's random swap of a top-k routing (``heta_route_swap``).
+
+    dense_idx: [B,k] int32 CUDA (the ``route`` output).  Returns (dense [B,k],
+    local [B,N-k], mask [B,N] uint8 or None); ``out`` may pass preallocated
+    (dense, local, mask), and dense may be dense_idx itself.
+    """
+    import torch
+    pd = _dev(dense_idx, torch.int32, "dense_idx", 2)
+    B, k = dense_idx.shape
+    if out is None:
+        dense = torch.empty((B, k), dtype=torch.int32, device=dense_idx.device)
+        local = torch.empty((B, N - k), dtype=torch.int32, device=dense_idx.device)
+        mask = (torch.empty((B, N), dtype=torch.uint8, device=dense_idx.device)
+                if want_mask else None)
+    else:
+        dense, local, mask = out
+    rc = load().heta_route_swap(pd if k > 0 else None, B, int(N), k, int(s),
+                                int(seed) & 0xFFFFFFFFFFFFFFFF, int(block),
+                                _opt(dense) if k > 0 else None, _opt(local) if k < N else None,
+                                _opt(mask), _opt(status), _stream())
+    _check(rc, "heta_route_swap")
+    return dense, local, mask
 
 
 def route_threshold(u, c: float, *, out=None, want_thresh=False, want_mask=False,

@@ -22,6 +22,10 @@ cudaError_t launch_route(const float *u, int B, int N, int k, int32_t *dense_idx
                          int32_t *local_idx, float *thresh, uint8_t *mask,
                          int32_t *status, cudaStream_t s);
 
+cudaError_t launch_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
+                              uint64_t seed, int block, int32_t *dense_out, int32_t *local_out,
+                              uint8_t *mask, int32_t *status, cudaStream_t st);
+
 cudaError_t launch_route_threshold(const float *u, int B, int N, double c, int32_t *counts,
                                    int32_t *dense_idx, int32_t *local_idx, double *thresh,
                                    uint8_t *mask, int32_t *status, cudaStream_t s);

@@ -14,6 +14,7 @@
 // are taken; a last pass compacts both index lists in increasing order with
 // warp ballots and writes them as contiguous runs.
 #include "heta_internal.cuh"
+#include "radix_select.cuh"
 
 namespace heta {
 namespace {
@@ -34,53 +35,6 @@ __device__ __forceinline__ float key_value(uint32_t key)
 {
     uint32_t b = (key & 0x80000000u) ? (key & 0x7fffffffu) : ~key;
     return __uint_as_float(b);
-}
-
-// The digit of the r-th largest key among those counted in hist[0..nbins)
-// (nbins = 1024 or 2048): *digit and *rank_in_digit (1-based) for the next
-// pass.  Bins are scanned from the top; every thread of the CTA calls this.
-__device__ __forceinline__ void find_digit(const uint32_t *hist, int nbins, uint32_t r,
-                                           uint32_t *warp_tot, uint32_t *s_digit,
-                                           uint32_t *s_rank)
-{
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = nbins / kThreads;  // 1 or 2 bins per thread, descending
-    uint32_t c[2] = {0u, 0u}, sum = 0u;
-    for (int j = 0; j < per; ++j) {
-        c[j] = hist[nbins - 1 - per * tid - j];
-        sum += c[j];
-    }
-    uint32_t incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    if (lane == 31) warp_tot[warp] = incl;
-    __syncthreads();
-    uint32_t wbefore = 0u;
-    {
-        const uint32_t wt = warp_tot[lane];
-        uint32_t wi = wt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t t = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += t;
-        }
-        wbefore = __shfl_sync(0xffffffffu, wi - wt, warp);
-    }
-    const uint32_t before = wbefore + incl - sum;
-    if (before < r && r <= before + sum) {
-        uint32_t acc = before;
-        for (int j = 0; j < per; ++j) {
-            if (acc < r && r <= acc + c[j]) {
-                *s_digit = (uint32_t)(nbins - 1 - per * tid - j);
-                *s_rank = r - acc;
-            }
-            acc += c[j];
-        }
-    }
-    __syncthreads();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -150,7 +104,7 @@ route_kernel(const float *__restrict__ u, int N, int k,
     // ---- 2. radix select of the k-th largest key: digits of 11, 11, 10 bits
     uint32_t kstar = 0xffffffffu, take = 0u;  // k == 0: nothing is dense
     if (k > 0) {
-        find_digit(hist, 2048, (uint32_t)k, warp_tot, &s_digit, &s_rank);
+        find_digit<kThreads>(hist, 2048, (uint32_t)k, warp_tot, &s_digit, &s_rank);
         const uint32_t d1 = s_digit, r1 = s_rank;
         for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
         __syncthreads();
@@ -167,7 +121,7 @@ route_kernel(const float *__restrict__ u, int N, int k,
             if ((key >> 21) == d1) atomicAdd(&hist[(key >> 10) & 2047u], 1u);
         }
         __syncthreads();
-        find_digit(hist, 2048, r1, warp_tot, &s_digit, &s_rank);
+        find_digit<kThreads>(hist, 2048, r1, warp_tot, &s_digit, &s_rank);
         const uint32_t p2 = (d1 << 11) | s_digit, r2 = s_rank;
         for (int i = tid; i < 1024; i += kThreads) hist[i] = 0u;
         __syncthreads();
@@ -183,7 +137,7 @@ route_kernel(const float *__restrict__ u, int N, int k,
             if ((key >> 10) == p2) atomicAdd(&hist[key & 1023u], 1u);
         }
         __syncthreads();
-        find_digit(hist, 1024, r2, warp_tot, &s_digit, &s_rank);
+        find_digit<kThreads>(hist, 1024, r2, warp_tot, &s_digit, &s_rank);
         kstar = (p2 << 10) | s_digit;
         take = s_rank;
     }
