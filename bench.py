@@ -428,6 +428,25 @@ def run_heta(args, info):
                "tokens_per_s": w.B * w.N / ((r_ms + a_ms) / 1e3)}
         del ws_t
 
+    # ---- the per-block random swap (Table 8: r = 7% of N) on this routing -----
+    swap = None
+    if not args.no_threshold_mode:
+        s_sw = heta.swap_count(w.N, kk, 0.07)
+        sw_d = torch.empty_like(dense)
+        sw_l = torch.empty_like(local)
+        heta.route(d_u, kk, out=(dense, local, None, None))
+        for _ in range(3):
+            heta.route_swap(dense, w.N, s_sw, 2024, 0, out=(sw_d, sw_l, None))
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 20
+        e0.record()
+        for blk in range(reps):
+            heta.route_swap(dense, w.N, s_sw, 2024, blk, out=(sw_d, sw_l, None))
+        e1.record()
+        torch.cuda.synchronize()
+        swap = {"r": 0.07, "s": s_sw, "us_per_block": 1e3 * e0.elapsed_time(e1) / reps}
+
     # ---- routing in throughput mode: 512 samples of this N in one launch -------
     route_tp = None
     if not args.no_route_throughput:
@@ -518,6 +537,7 @@ def run_heta(args, info):
         "window_sweep": win_sweep,
         "threshold_mode": thr,
         "route_throughput": route_tp,
+        "route_swap": swap,
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu, "clocks": sampler.summary(),
     }
