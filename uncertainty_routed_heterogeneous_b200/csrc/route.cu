@@ -38,7 +38,7 @@ __device__ __forceinline__ float key_value(uint32_t key)
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-route_kernel(const float *__restrict__ u, int N, int k,
+route_kernel(const float *__restrict__ u, int B, int N, int k,
              int32_t *__restrict__ dense_idx, int32_t *__restrict__ local_idx,
              float *__restrict__ thresh, uint8_t *__restrict__ mask,
              int32_t *status)
@@ -52,8 +52,15 @@ route_kernel(const float *__restrict__ u, int N, int k,
     __shared__ int s_nan;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x;
+    // samples b = blockIdx.x, + gridDim.x, ...: while one is processed, the
+    // next one's u is pulled into L2
+    for (int b = blockIdx.x; b < B; b += gridDim.x) {
     const float *ub = u + (size_t)b * N;
+    if (b + (int)gridDim.x < B) {
+        const char *nx = reinterpret_cast<const char *>(ub + (size_t)gridDim.x * N);
+        for (size_t off = (size_t)tid * 128; off < (size_t)N * 4; off += (size_t)kThreads * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(nx + off));
+    }
     if (tid == 0) s_nan = 0;
     for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
     __syncthreads();
@@ -109,12 +116,21 @@ route_kernel(const float *__restrict__ u, int N, int k,
         for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
         __syncthreads();
         const uint4 *keys4 = reinterpret_cast<const uint4 *>(keys);
-        for (int v = tid; v < (N >> 2); v += kThreads) {
-            const uint4 q = keys4[v];
-            if ((q.x >> 21) == d1) atomicAdd(&hist[(q.x >> 10) & 2047u], 1u);
-            if ((q.y >> 21) == d1) atomicAdd(&hist[(q.y >> 10) & 2047u], 1u);
-            if ((q.z >> 21) == d1) atomicAdd(&hist[(q.z >> 10) & 2047u], 1u);
-            if ((q.w >> 21) == d1) atomicAdd(&hist[(q.w >> 10) & 2047u], 1u);
+        // (the keys still in the running are few: one vote per four keys
+        // skips the counting where a warp holds none)
+        // (the loop runs warp-uniformly: the vote needs every lane)
+        for (int vb = tid - lane; vb < (N >> 2); vb += kThreads) {
+            const int v = vb + lane;
+            const uint4 q = v < (N >> 2) ? keys4[v] : make_uint4(0u, 0u, 0u, 0u);
+            const bool in = v < (N >> 2);
+            const bool m0 = in && (q.x >> 21) == d1, m1 = in && (q.y >> 21) == d1;
+            const bool m2 = in && (q.z >> 21) == d1, m3 = in && (q.w >> 21) == d1;
+            if (__any_sync(0xffffffffu, m0 | m1 | m2 | m3)) {
+                if (m0) atomicAdd(&hist[(q.x >> 10) & 2047u], 1u);
+                if (m1) atomicAdd(&hist[(q.y >> 10) & 2047u], 1u);
+                if (m2) atomicAdd(&hist[(q.z >> 10) & 2047u], 1u);
+                if (m3) atomicAdd(&hist[(q.w >> 10) & 2047u], 1u);
+            }
         }
         for (int i = 4 * (N >> 2) + tid; i < N; i += kThreads) {
             const uint32_t key = keys[i];
@@ -125,12 +141,18 @@ route_kernel(const float *__restrict__ u, int N, int k,
         const uint32_t p2 = (d1 << 11) | s_digit, r2 = s_rank;
         for (int i = tid; i < 1024; i += kThreads) hist[i] = 0u;
         __syncthreads();
-        for (int v = tid; v < (N >> 2); v += kThreads) {
-            const uint4 q = keys4[v];
-            if ((q.x >> 10) == p2) atomicAdd(&hist[q.x & 1023u], 1u);
-            if ((q.y >> 10) == p2) atomicAdd(&hist[q.y & 1023u], 1u);
-            if ((q.z >> 10) == p2) atomicAdd(&hist[q.z & 1023u], 1u);
-            if ((q.w >> 10) == p2) atomicAdd(&hist[q.w & 1023u], 1u);
+        for (int vb = tid - lane; vb < (N >> 2); vb += kThreads) {
+            const int v = vb + lane;
+            const uint4 q = v < (N >> 2) ? keys4[v] : make_uint4(0u, 0u, 0u, 0u);
+            const bool in = v < (N >> 2);
+            const bool m0 = in && (q.x >> 10) == p2, m1 = in && (q.y >> 10) == p2;
+            const bool m2 = in && (q.z >> 10) == p2, m3 = in && (q.w >> 10) == p2;
+            if (__any_sync(0xffffffffu, m0 | m1 | m2 | m3)) {
+                if (m0) atomicAdd(&hist[q.x & 1023u], 1u);
+                if (m1) atomicAdd(&hist[q.y & 1023u], 1u);
+                if (m2) atomicAdd(&hist[q.z & 1023u], 1u);
+                if (m3) atomicAdd(&hist[q.w & 1023u], 1u);
+            }
         }
         for (int i = 4 * (N >> 2) + tid; i < N; i += kThreads) {
             const uint32_t key = keys[i];
@@ -202,26 +224,69 @@ route_kernel(const float *__restrict__ u, int N, int k,
     int32_t *dout = dense_idx + (size_t)b * k;
     int32_t *lout = local_idx + (size_t)b * (N - k);
     uint8_t *mout = mask ? mask + (size_t)b * N : nullptr;
-    for (int base = seg_lo; base < seg_hi; base += 32) {
-        const int i = base + lane;
-        const bool valid = i < seg_hi;
-        const uint32_t key = valid ? keys[i] : 0u;
-        const bool gt = valid && key > kstar;
-        const bool eq = valid && key == kstar;
-        const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-        const uint32_t eq_rank = re + __popc(eq_mask & lt);
-        const bool dense = gt || (eq && eq_rank < take);
-        const unsigned d_mask = __ballot_sync(0xffffffffu, dense);
-        const uint32_t pos = rd + __popc(d_mask & lt);  // dense tokens before i
-        // the select makes |dense| == k exactly; the bounds only guard memory
-        if (dense) {
-            if (pos < (uint32_t)k) dout[pos] = i;
-        } else if (valid && (uint32_t)i - pos < (uint32_t)(N - k)) {
-            lout[i - pos] = i;
+    // 128 tokens per warp step, four consecutive ones per lane: token
+    // t0 + e (e < 4) is dense-ranked by the lanes before it (one ballot per e)
+    // and by the lane's own earlier tokens
+    for (int base = seg_lo; base < seg_hi; base += 128) {
+        const int t0 = base + 4 * lane;
+        uint32_t key[4];
+        if (t0 + 3 < seg_hi) {
+            const uint4 q = *reinterpret_cast<const uint4 *>(keys + t0);
+            key[0] = q.x;
+            key[1] = q.y;
+            key[2] = q.z;
+            key[3] = q.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) key[e] = t0 + e < seg_hi ? keys[t0 + e] : 0u;
         }
-        if (mout && valid) mout[i] = dense ? 0 : 1;
-        rd += __popc(d_mask);
-        re += __popc(eq_mask);
+        bool valid[4], dense[4];
+        bool any_eq = false;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            valid[e] = t0 + e < seg_hi;
+            dense[e] = valid[e] && key[e] > kstar;
+            any_eq |= valid[e] && key[e] == kstar;
+        }
+        if (__any_sync(0xffffffffu, any_eq)) {
+            // keys equal to K*: the first `take` of them in token order
+            uint32_t before = re, own = 0;
+            unsigned em[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                em[e] = __ballot_sync(0xffffffffu, valid[e] && key[e] == kstar);
+                before += __popc(em[e] & lt);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool eq = valid[e] && key[e] == kstar;
+                dense[e] = dense[e] || (eq && before + own < take);
+                own += eq;
+                re += __popc(em[e]);
+            }
+        }
+        unsigned dm[4];
+        uint32_t pos = rd;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            dm[e] = __ballot_sync(0xffffffffu, dense[e]);
+            pos += __popc(dm[e] & lt);
+        }
+        // one store per token into whichever list holds it; the select makes
+        // |dense| == k exactly, the bounds only guard memory
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint32_t t = (uint32_t)(t0 + e);
+            const uint32_t slot = dense[e] ? pos : t - pos;
+            const uint32_t cap = dense[e] ? (uint32_t)k : (uint32_t)(N - k);
+            int32_t *const list = dense[e] ? dout : lout;
+            if (valid[e] && slot < cap) list[slot] = (int32_t)t;
+            if (mout && valid[e]) mout[t] = dense[e] ? 0 : 1;
+            pos += dense[e];
+            rd += __popc(dm[e]);
+        }
+    }
+    __syncthreads();  // shared memory is reused by the next sample
     }
 }
 
@@ -236,8 +301,11 @@ cudaError_t launch_route(const float *u, int B, int N, int k, int32_t *dense_idx
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(sizeof(uint32_t) * kRouteMaxN));
     if (e != cudaSuccess) return e;
-    route_kernel<<<B, kThreads, smem, s>>>(u, N, k, dense_idx, local_idx, thresh,
-                                           mask, status);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    route_kernel<<<B < sms ? B : sms, kThreads, smem, s>>>(u, B, N, k, dense_idx, local_idx,
+                                                         thresh, mask, status);
     return cudaGetLastError();
 }
 
