@@ -12,10 +12,12 @@
 //               (all N keys, or half of them when the host splits the key
 //               range to balance the SMs; the second half to finish merges
 //               the other's partial result -- no CTA ever waits on another).
-//   LOCAL item: two 2x8x8 query boxes of the latent grid; each box streams
-//               the 1x8x16-key K/V sub-tiles that cover its rows' windows,
-//               with a per-element window mask.  Rows whose token is dense
-//               are computed but not stored.
+//   LOCAL item: two 128-token query boxes of the latent grid (2x8x8 for
+//               small windows; the planner picks the shape whose K/V covers
+//               hold the fewest keys, e.g. 8x4x4 for an 11^3 window); each
+//               box streams the 1x8x16-key K/V sub-tiles that cover its rows'
+//               windows, with a per-element window mask.  Rows whose token
+//               is dense are computed but not stored.
 // Per CTA (one per SM): a TMA producer warp fills a shared-memory ring of K/V
 // tiles (128-byte swizzle) and loads LOCAL query boxes; one thread issues
 // tcgen05.mma with fp32 accumulators in TMEM (S = Q K^T, O += P V with P read
@@ -50,7 +52,8 @@ constexpr float kRescaleLog2 = 8.0f;    // rescale O only when the max grows > 2
 constexpr int kQueue = 4;               // work-item queue depth
 
 // query box (LOCAL) and key sub-tile
-constexpr int kBoxT = 2, kBoxH = 8, kBoxW = 8;
+// (the query box is planned per call among shapes of 128 tokens, see
+// plan_attention; the key sub-tile is fixed)
 constexpr int kKvH = 8, kKvW = 16;
 
 enum { DENSE = 0, LOCAL = 1 };
@@ -72,6 +75,7 @@ struct Params {
     // DENSE items
     int tiles_d, pairs_d, nsplit, n_kv_d, kv_per_split, n_dense_items;
     // LOCAL items
+    int box_t, box_h, box_w;
     int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
     int total_items;
     // scratch
@@ -200,9 +204,9 @@ __device__ __forceinline__ Box local_box(const Params &p, int box)
     x.active = box < p.tiles_l;
     const int bb = x.active ? box : 0;
     const int bw = bb % p.nbw, bh = (bb / p.nbw) % p.nbh, bt = bb / (p.nbw * p.nbh);
-    x.t0 = bt * kBoxT;
-    x.h0 = bh * kBoxH;
-    x.w0 = bw * kBoxW;
+    x.t0 = bt * p.box_t;
+    x.h0 = bh * p.box_h;
+    x.w0 = bw * p.box_w;
     x.tlo = min(wstart(x.t0, p.Tg, p.wt), p.Tg - p.nkt);
     x.hlo = min(wstart(x.h0, p.Hg, p.wh), max(0, p.Hg - p.nkh * kKvH));
     x.wlo = min(wstart(x.w0, p.Wg, p.ww), max(0, p.Wg - p.nkw * kKvW));
@@ -633,9 +637,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 const Box x = local_box(p, it.tile[t]);
                 if (!x.active) continue;
                 const int lo_tok = (x.t0 * p.Hg + x.h0) * p.Wg + x.w0;
-                const int hi_tok = (min(x.t0 + kBoxT, p.Tg) - 1) * HW +
-                                   (min(x.h0 + kBoxH, p.Hg) - 1) * p.Wg +
-                                   min(x.w0 + kBoxW, p.Wg) - 1;
+                const int hi_tok = (min(x.t0 + p.box_t, p.Tg) - 1) * HW +
+                                   (min(x.h0 + p.box_h, p.Hg) - 1) * p.Wg +
+                                   min(x.w0 + p.box_w, p.Wg) - 1;
                 // first position with dense_idx >= lo_tok (32-ary search)
                 int lo = 0, hi = it.kb;
                 while (hi - lo > 32) {
@@ -659,9 +663,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                     if (v <= hi_tok) {
                         const int tt = v / HW - x.t0, hh = (v / p.Wg) % p.Hg - x.h0,
                                   ww = v % p.Wg - x.w0;
-                        if (tt >= 0 && tt < kBoxT && hh >= 0 && hh < kBoxH && ww >= 0 &&
-                            ww < kBoxW)
-                            sh.no_store[t][(tt * kBoxH + hh) * kBoxW + ww] = 1;
+                        if (tt >= 0 && tt < p.box_t && hh >= 0 && hh < p.box_h && ww >= 0 &&
+                            ww < p.box_w)
+                            sh.no_store[t][(tt * p.box_h + hh) * p.box_w + ww] = 1;
                     }
                     if (__ballot_sync(0xffffffffu, v <= hi_tok) != 0xffffffffu) break;
                 }
@@ -714,8 +718,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 if (r == 0) mbar_arrive(smem_addr(&sh.q_full[t]));
             } else {
                 bx = local_box(p, tile);
-                const int qt = bx.t0 + r / (kBoxH * kBoxW), qh = bx.h0 + (r / kBoxW) % kBoxH,
-                          qw = bx.w0 + r % kBoxW;
+                const int qt = bx.t0 + r / (p.box_h * p.box_w),
+                          qh = bx.h0 + (r / p.box_w) % p.box_h, qw = bx.w0 + r % p.box_w;
                 row_valid = bx.active && qt < p.Tg && qh < p.Hg && qw < p.Wg;
                 token = (qt * p.Hg + qh) * p.Wg + qw;
                 qs_t = wstart(min(qt, p.Tg - 1), p.Tg, p.wt);
@@ -947,14 +951,38 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     pl.nsplit = (k > 0 && pairs_total < 4 * kPlanSMs && pl.n_kv_d >= 16) ? 2 : 1;
     pl.kv_per_split = (pl.n_kv_d + pl.nsplit - 1) / pl.nsplit;
     pl.n_dense_items = (int)(pairs_total * pl.nsplit);
-    const int nbt = (Tg + kBoxT - 1) / kBoxT;
-    pl.nbh = (Hg + kBoxH - 1) / kBoxH;
-    pl.nbw = (Wg + kBoxW - 1) / kBoxW;
+    // LOCAL query box: of the 128-token shapes below, the one whose boxes'
+    // K/V covers hold the fewest keys in all (a box's cover spans the union of
+    // its rows' windows, rounded up to whole 1x8x16 key sub-tiles); ties keep
+    // the earlier shape.  Small windows take 2x8x8, an 11^3 window 8x4x4.
+    {
+        static const int shapes[][3] = {{2, 8, 8}, {4, 4, 8}, {4, 8, 4}, {8, 4, 4},
+                                        {2, 4, 16}, {1, 8, 16}, {8, 8, 2}};
+        int64_t best = -1;
+        for (const auto &sh : shapes) {
+            const int bt = sh[0], bh = sh[1], bw = sh[2];
+            const int64_t boxes = (int64_t)((Tg + bt - 1) / bt) * ((Hg + bh - 1) / bh) *
+                                  ((Wg + bw - 1) / bw);
+            const int nkt = min(bt + wt - 1, Tg);
+            const int nkh = (min(bh + wh - 1, Hg) + kKvH - 1) / kKvH;
+            const int nkw = (min(bw + ww - 1, Wg) + kKvW - 1) / kKvW;
+            const int64_t cost = ((boxes + 1) / 2) * nkt * nkh * nkw;
+            if (best < 0 || cost < best) {
+                best = cost;
+                pl.box_t = bt;
+                pl.box_h = bh;
+                pl.box_w = bw;
+            }
+        }
+    }
+    const int nbt = (Tg + pl.box_t - 1) / pl.box_t;
+    pl.nbh = (Hg + pl.box_h - 1) / pl.box_h;
+    pl.nbw = (Wg + pl.box_w - 1) / pl.box_w;
     pl.tiles_l = nbt * pl.nbh * pl.nbw;
     pl.pairs_l = (pl.tiles_l + 1) / 2;
-    pl.nkt = min(kBoxT + wt - 1, Tg);
-    pl.nkh = (min(kBoxH + wh - 1, Hg) + kKvH - 1) / kKvH;
-    pl.nkw = (min(kBoxW + ww - 1, Wg) + kKvW - 1) / kKvW;
+    pl.nkt = min(pl.box_t + wt - 1, Tg);
+    pl.nkh = (min(pl.box_h + wh - 1, Hg) + kKvH - 1) / kKvH;
+    pl.nkw = (min(pl.box_w + ww - 1, Wg) + kKvW - 1) / kKvW;
     pl.n_kv_l = pl.nkt * pl.nkh * pl.nkw;
     pl.n_local_items = (k < N || per_sample_counts) ? B * H * pl.pairs_l : 0;
     pl.total_items = pl.n_dense_items + pl.n_local_items;
@@ -983,6 +1011,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.tiles_d = pl.tiles_d; p.pairs_d = pl.pairs_d; p.nsplit = pl.nsplit;
     p.n_kv_d = pl.n_kv_d; p.kv_per_split = pl.kv_per_split; p.n_dense_items = pl.n_dense_items;
+    p.box_t = pl.box_t; p.box_h = pl.box_h; p.box_w = pl.box_w;
     p.tiles_l = pl.tiles_l; p.pairs_l = pl.pairs_l; p.nbh = pl.nbh; p.nbw = pl.nbw;
     p.nkt = pl.nkt; p.nkh = pl.nkh; p.nkw = pl.nkw; p.n_kv_l = pl.n_kv_l;
     p.n_local_items = pl.n_local_items; p.total_items = pl.total_items;
@@ -998,7 +1027,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     if (!map_rows(&k3, a.K, BH, a.N, D) || !map_rows(&v3, a.V, BH, a.N, D) ||
         !map_grid(&k5, a.K, BH, a.Tg, a.Hg, a.Wg, D, 1, kKvH, kKvW) ||
         !map_grid(&v5, a.V, BH, a.Tg, a.Hg, a.Wg, D, 1, kKvH, kKvW) ||
-        !map_grid(&q5, a.Q, BH, a.Tg, a.Hg, a.Wg, D, kBoxT, kBoxH, kBoxW))
+        !map_grid(&q5, a.Q, BH, a.Tg, a.Hg, a.Wg, D, pl.box_t, pl.box_h, pl.box_w))
         return cudaErrorInvalidValue;
 
     cudaError_t e = cudaMemsetAsync(workspace, 0, pl.zero_bytes, s);
