@@ -280,6 +280,21 @@ HETA_API heta_status heta_uncertainty(const uint16_t *X, const float *w, float b
                              int B, int N, int C, float *u_out,
                              int32_t *status_dev, void *stream);
 
+/*
+ * heta_selftest_wait_timeout -- test hook (the paper has no counterpart):
+ * runs the bounded-wait path every kernel of this library uses, on purpose.
+ * One small kernel: warp 0 waits on a barrier that nothing completes until
+ * limit_ns of wall time have passed, raises the CTA's abort flag and writes
+ * HETA_ERR_TIMEOUT to *status_dev (atomic max); warp 1 waits on another such
+ * barrier with a 5 s limit and must be released by the flag.  If
+ * elapsed_ns_dev is not NULL it receives the kernel's wall time (device
+ * uint64).  Nothing faults and nothing is left in flight: the context stays
+ * usable.  Requires 0 < limit_ns <= 10 s and status_dev (device int32).
+ */
+HETA_API heta_status heta_selftest_wait_timeout(uint64_t limit_ns, int32_t *status_dev,
+                                                unsigned long long *elapsed_ns_dev,
+                                                void *stream);
+
 #ifdef __cplusplus
 }
 #endif

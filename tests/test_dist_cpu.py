@@ -53,3 +53,36 @@ def test_head_ranges_partition(H, world):
         lo, hi = D.head_range(H, world, r)
         seen += list(range(lo, hi))
     assert seen == list(range(H))
+
+
+def _worker_one_dies(rank, world, port, q):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    info = D.rank_info()
+    D.init("gloo", info, timeout_s=5)
+    if rank == 1:
+        # a rank that fails between steps: it leaves without its next collective
+        os._exit(3)
+    import time
+    t0 = time.monotonic()
+    try:
+        D.barrier(info)
+        D.max_over_ranks(1.0, info)
+        q.put(("no error", time.monotonic() - t0))
+    except Exception as e:  # the surviving rank learns of it as an error, not a hang
+        q.put((type(e).__name__, time.monotonic() - t0))
+
+
+def test_a_rank_that_dies_ends_the_others_collective_with_an_error():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker_one_dies, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    what, secs = q.get(timeout=120)
+    for p in procs:
+        p.join(60)
+    assert what != "no error"
+    assert secs < 60
+    assert procs[1].exitcode == 3

@@ -66,6 +66,8 @@ def load():
     lib.heta_attention.restype = i
     lib.heta_uncertainty.argtypes = [vp, vp, f, i, i, i, vp, vp, vp]
     lib.heta_uncertainty.restype = i
+    lib.heta_selftest_wait_timeout.argtypes = [ctypes.c_uint64, vp, vp, vp]
+    lib.heta_selftest_wait_timeout.restype = i
     lib.heta_route_swap.argtypes = [vp, i, i, i, i, ctypes.c_uint64, i, vp, vp, vp, vp, vp]
     lib.heta_route_swap.restype = i
     lib.heta_route_threshold.argtypes = [vp, i, i, d, vp, vp, vp, vp, vp, vp, vp]
@@ -140,6 +142,17 @@ def route(u, k: int, *, out=None, want_thresh=False, want_mask=False, status=Non
                            _opt(status), _stream())
     _check(rc, "heta_route")
     return dense, local, thresh, mask
+
+
+def selftest_wait_timeout(limit_ns: int, status, elapsed=None):
+    """Runs the library's bounded-wait path into a timeout on purpose
+    (``heta_selftest_wait_timeout``): status (int32 CUDA) receives
+    HETA_ERR_TIMEOUT; elapsed (int64 CUDA, optional) the kernel's wall time."""
+    import torch
+    ps = _dev(status, torch.int32, "status")
+    pe = _dev(elapsed, torch.int64, "elapsed") if elapsed is not None else None
+    _check(load().heta_selftest_wait_timeout(int(limit_ns), ps, pe, _stream()),
+           "heta_selftest_wait_timeout")
 
 
 def swap_count(N: int, k: int, r: float) -> int:
