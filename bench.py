@@ -48,6 +48,10 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["heta", "reference"], default="heta")
     p.add_argument("--workload", default=W.WAN21.name, choices=sorted(W.ALL))
+    p.add_argument("--rho", type=float, default=None,
+                   help="dense fraction (default: the workload's own, 0.2)")
+    p.add_argument("--window", default=None,
+                   help="local window as TxHxW, odd sizes (default: the workload's own)")
     p.add_argument("--cpu-tokens", type=int, default=1536,
                    help="tokens in the oracle's bounded CPU sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -59,9 +63,27 @@ def parse_args():
                    help="skip timing the paper's mu + c*sigma routing (c = 0.9)")
     p.add_argument("--no-route-throughput", action="store_true",
                    help="skip timing heta_route on 512 samples in one launch")
+    p.add_argument("--nvtx", action="store_true",
+                   help="mark route / attention / head of every step with NVTX ranges")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="minimum host time the cpu_baseline oracle sample runs for")
     return p.parse_args()
+
+
+def chosen_workload(args):
+    """The named workload, with --rho / --window applied (a renamed copy)."""
+    import dataclasses
+    w = W.ALL[args.workload]
+    if args.rho is not None:
+        if not 0.0 <= args.rho <= 1.0:
+            raise SystemExit("--rho must lie in [0, 1]")
+        w = dataclasses.replace(w, name="%s-rho%g" % (w.name, args.rho), rho=args.rho)
+    if args.window is not None:
+        win = tuple(int(x) for x in args.window.lower().split("x"))
+        if len(win) != 3 or any(x < 1 or x % 2 == 0 for x in win):
+            raise SystemExit("--window takes three odd sizes, e.g. 11x11x11")
+        w = dataclasses.replace(w, name="%s-win%s" % (w.name, args.window), win=win)
+    return w
 
 
 def load_peaks():
@@ -188,7 +210,7 @@ def run_reference(args, info):
     import oracle
     if info.rank != 0:
         return 0
-    w = W.ALL[args.workload]
+    w = chosen_workload(args)
     s = OracleSample(w, n_tokens=max(16, args.cpu_tokens // 6))
     for _ in range(args.warmup):
         s.step()
@@ -275,7 +297,7 @@ def run_heta(args, info):
     dev = torch.device("cuda", info.local_rank)
     D.init("nccl", info, timeout_s=300)
     heta.load()
-    base = W.ALL[args.workload]
+    base = chosen_workload(args)
     w = D.rank_workload(base, info.rank)
 
     # ---- inputs: host (pinned) and resident device copies -------------------
@@ -304,18 +326,30 @@ def run_heta(args, info):
     h_unext = torch.empty(u_next.shape, dtype=torch.float32).pin_memory()
     torch.cuda.synchronize()
 
+    nvtx = torch.cuda.nvtx if args.nvtx else None
+
     def step(ev=None):
         if ev is not None:
             ev[0].record()
+        if nvtx:
+            nvtx.range_push("heta_route")
         heta.route(d_u, kk, out=(dense, local, None, None))
         if ev is not None:
             ev[1].record()
+        if nvtx:
+            nvtx.range_pop()
+            nvtx.range_push("heta_attention")
         heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense, out=out, workspace=ws)
         if ev is not None:
             ev[2].record()
+        if nvtx:
+            nvtx.range_pop()
+            nvtx.range_push("heta_uncertainty")
         heta.uncertainty(d_X, d_w, 0.0, out=u_next)
         if ev is not None:
             ev[3].record()
+        if nvtx:
+            nvtx.range_pop()
 
     # route, the persistent attention kernel, the head (plus one workspace memset)
     launches_per_step = 3

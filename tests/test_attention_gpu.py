@@ -71,7 +71,10 @@ def test_multi_tile_all_rows(gpu_lib, w, rho):
 @pytest.mark.parametrize("name", ["wan2.1-1.3b-21x30x52", "wan2.2-5b-31x22x40",
                                   "wan2.1-1.3b-batched-b2"])
 def test_full_size_sampled_rows(gpu_lib, name):
-    run(gpu_lib, W.ALL[name], n_sample=1500)
+    """4096 random rows per head on average, plus every border-clamped window
+    class and the first and last dense rows of the first and last head."""
+    w = W.ALL[name]
+    run(gpu_lib, w, n_sample=4096 * w.B * w.H)
 
 
 @pytest.mark.parametrize("rho", [0.05, 0.5])
