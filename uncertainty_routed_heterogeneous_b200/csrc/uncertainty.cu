@@ -48,10 +48,12 @@ __device__ __forceinline__ float softplus(float z)
     return z > 0.f ? z + log1pf(expf(-z)) : log1pf(expf(z));
 }
 
-// UNROLL row-chunks of 8 elements are loaded before any is consumed, so each
-// lane keeps UNROLL 16-byte loads in flight.
+// A warp walks its rows in slices of 32 * UNROLL 16-byte chunks (one slice
+// is a whole row at C <= 256 * UNROLL).  The next slice's UNROLL loads per
+// lane are issued before the current slice is consumed, so loads stay in
+// flight through the arithmetic, the shuffle reduction and the store.
 template <int UNROLL>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 uncertainty_kernel(const uint16_t *__restrict__ X, const float *__restrict__ w,
                    float bias, int64_t rows, int C, float *__restrict__ u)
 {
@@ -62,26 +64,44 @@ uncertainty_kernel(const uint16_t *__restrict__ X, const float *__restrict__ w,
     const int lane = threadIdx.x & 31;
     const int chunks = C >> 3;  // 8 bf16 per 16-byte chunk
     const int64_t nwarps = (int64_t)gridDim.x * kWarps;
-    for (int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); row < rows;
-         row += nwarps) {
-        const uint4 *xr = reinterpret_cast<const uint4 *>(X + row * C);
-        float acc = 0.f;
-        for (int c0 = 0; c0 < chunks; c0 += 32 * UNROLL) {
-            uint4 v[UNROLL];
+    int64_t row = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    int c0 = 0;
+    auto load = [&](int64_t r, int cb, uint4 (&v)[UNROLL]) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(X + r * C);
 #pragma unroll
-            for (int j = 0; j < UNROLL; ++j) {
-                const int c = c0 + j * 32 + lane;
-                v[j] = c < chunks ? ld_stream(xr + c) : make_uint4(0u, 0u, 0u, 0u);
-            }
-#pragma unroll
-            for (int j = 0; j < UNROLL; ++j) {
-                const int c = c0 + j * 32 + lane;
-                if (c < chunks) acc += dot8(v[j], ws + 8 * c);
-            }
+        for (int j = 0; j < UNROLL; ++j) {
+            const int c = cb + j * 32 + lane;
+            v[j] = c < chunks ? ld_stream(xr + c) : make_uint4(0u, 0u, 0u, 0u);
         }
+    };
+    uint4 v[UNROLL];
+    if (row < rows) load(row, 0, v);
+    float acc = 0.f;
+    while (row < rows) {
+        // the slice after this one
+        int64_t nrow = row;
+        int nc0 = c0 + 32 * UNROLL;
+        if (nc0 >= chunks) {
+            nrow = row + nwarps;
+            nc0 = 0;
+        }
+        uint4 vn[UNROLL];
+        if (nrow < rows) load(nrow, nc0, vn);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) u[row] = softplus(acc + bias);
+        for (int j = 0; j < UNROLL; ++j) {
+            const int c = c0 + j * 32 + lane;
+            if (c < chunks) acc += dot8(v[j], ws + 8 * c);
+        }
+        if (nrow != row) {  // the row is complete
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (lane == 0) u[row] = softplus(acc + bias);
+            acc = 0.f;
+        }
+        row = nrow;
+        c0 = nc0;
+#pragma unroll
+        for (int j = 0; j < UNROLL; ++j) v[j] = vn[j];
     }
 }
 
