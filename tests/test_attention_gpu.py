@@ -107,3 +107,41 @@ def test_window_cube_all_rows(gpu_lib, n, rho):
 @pytest.mark.parametrize("n", W.WINDOW_CUBES)
 def test_window_cube_full_size_sampled_rows(gpu_lib, n):
     run(gpu_lib, W.window_cube(n), n_sample=1000)
+
+
+# Degenerate cases of the method: a single dense row, all but one row dense,
+# a one-frame grid, a 1x1x1 window (each local row attends to itself only, so
+# its output is its own v), one head and three samples.
+@pytest.mark.parametrize("case", ["k1", "k_n_minus_1", "one_frame", "win111", "b3_h1"])
+def test_degenerate_cases(gpu_lib, case):
+    import torch
+    heta = gpu_lib
+    base = W.scaled(W.WAN21, H=2, grid=(3, 10, 14), win=(3, 5, 5), u_kind="uniform",
+                    u_seeds=(21,))
+    if case == "k1":
+        w, kk = base, 1
+    elif case == "k_n_minus_1":
+        w, kk = base, base.N - 1
+    elif case == "one_frame":
+        w = dataclasses.replace(base, grid=(1, 12, 20), win=(1, 7, 9))
+        kk = heta.dense_count(w.N, 0.2)
+    elif case == "win111":
+        w = dataclasses.replace(base, win=(1, 1, 1))
+        kk = heta.dense_count(w.N, 0.2)
+    else:
+        w = dataclasses.replace(base, B=3, H=1, u_seeds=(21, 22, 23))
+        kk = heta.dense_count(w.N, 0.3)
+    w = dataclasses.replace(w, name="degenerate-" + case)
+    rho = kk / w.N
+    mx, mean = run(heta, w, rho=rho)
+    if case == "win111":
+        # local rows reproduce their own value vector (bf16 in, bf16 out)
+        q, k, v = W.make_qkv(w)
+        Qd, Kd, Vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+        dense, local, _, _ = heta.route(to_dev(W.make_u(w)), kk)
+        out = heta.attention(Qd, Kd, Vd, w.grid, w.win, dense)
+        torch.cuda.synchronize()
+        loc = local.cpu().numpy()[0]
+        got = from_dev_bf16(out)[0][:, loc]
+        want = W.bf16_to_f32(v)[0][:, loc]
+        assert np.array_equal(got, want)

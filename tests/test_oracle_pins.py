@@ -572,3 +572,16 @@ def test_head_special_cases():
     assert abs(oracle.uncertainty(big, np.ones(1, np.float32))[0, 0] - 60.0) < 1e-12
     small = np.full((1, 1, 1), -60.0, np.float32)
     assert abs(oracle.uncertainty(small, np.ones(1, np.float32))[0, 0] - math.exp(-60)) < 1e-36
+
+
+def test_window_111_local_rows_return_their_own_value():
+    """A 1x1x1 neighbourhood holds only the token itself (R3): its softmax has
+    one term, so a local row's output is its own v exactly."""
+    rng = np.random.default_rng(2)
+    grid, win = (2, 4, 5), (1, 1, 1)
+    N = 40
+    q, k, v = (rng.standard_normal((1, 2, N, 8)).astype(np.float32) for _ in range(3))
+    dense = np.array([[3, 17, 30]], np.int32)
+    out = oracle.attention(q, k, v, grid, win, dense)
+    loc = np.setdiff1d(np.arange(N), dense[0])
+    assert np.array_equal(out[0][:, loc], v[0][:, loc].astype(np.float64))
