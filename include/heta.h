@@ -162,10 +162,11 @@ HETA_API heta_status heta_route_threshold(const float *u, int B, int N, double c
  * needs for these sizes (host-only; touches no device).
  *
  * The scratch holds the work-item counter of the persistent kernel and, when
- * the dense rows' key range is split in two to keep all SMs busy, the
- * partial results the two halves merge (fp32, about 1 KB per dense row and
- * half for d = 64).  At the Wan2.1-1.3B shape with rho = 0.2 that is about
- * 83 MB; when no split is needed it is 256 bytes.  Same argument rules as
+ * the pairs of dense query tiles of the last, partial wave of work are cut
+ * into 2..8 key ranges to keep all SMs busy, the partial results those
+ * ranges merge (fp32, about 1 KB per row and range, half for d = 64; at most
+ * ~19 MB).  At the Wan2.1-1.3B shape with rho = 0.2 that is about 17 MB;
+ * when the dense pairs make whole waves it is 256 bytes.  Same argument rules as
  * heta_attention; *bytes is only written on HETA_OK.
  */
 HETA_API heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg,

@@ -179,15 +179,20 @@ def test_flop_model_matches_the_papers_reduction():
 
 
 def test_workspace_size(lib):
-    """Counter-only scratch when the dense pairs fill the SMs; a split merge buffer
-    when they do not (Wan2.1 shape at rho = 0.2)."""
-    full = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), 32760)
-    assert full == 256
+    """Whole waves of dense pairs run unsplit and need no scratch beyond the
+    work counter; the pairs of the last, partial wave are cut into 2..8 key
+    ranges whose fp32 partials the workspace holds."""
+    # rho = 0.2: 312 pairs = 2 waves of 148 + 16 pairs cut in 8 (148 // 16 = 9 -> 8)
     k = heta.dense_count(32760, 0.2)
     part = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k)
-    pairs = 12 * (((k + 127) // 128 + 1) // 2)
-    assert part >= pairs * 2 * 2 * 128 * (128 * 4 + 8)
-    assert part < 100 * 2 ** 20
+    assert part >= 16 * 8 * 2 * 128 * (128 * 4 + 8)
+    assert part < 20 * 2 ** 20
+    # exactly whole waves: 148 pairs of 2 tiles -> no split, counter only
+    k148 = 148 * 256
+    w = heta.attention_workspace_size(1, 1, 128, (37, 32, 32), (3, 9, 9), k148)
+    assert w == 256
+    # no dense rows, or too few key tiles to split: counter only
     assert heta.attention_workspace_size(1, 2, 64, (4, 8, 8), (3, 3, 3), 0) == 256
+    assert heta.attention_workspace_size(1, 2, 64, (4, 8, 8), (3, 3, 3), 200) == 256
     with pytest.raises(heta.HetaError):
         heta.attention_workspace_size(1, 2, 96, (4, 8, 8), (3, 3, 3), 10)

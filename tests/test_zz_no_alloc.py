@@ -67,13 +67,16 @@ def test_noalloc_matches_workspace_entry_point(gpu_lib, grid, win, rho, H, d):
 
 
 def test_noalloc_refuses_sizes_beyond_its_array(gpu_lib):
-    """The Wan2.1-shaped call at rho = 0.2 needs ~83 MB of scratch: refused up front."""
+    """A call whose scratch would not fit the 16 MiB array is refused up front,
+    before anything is launched (the pointers below are never touched)."""
     heta = gpu_lib
     fn = _noalloc(heta.load())
-    k = heta.dense_count(32760, 0.2)
-    need = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k)
-    assert need > 16 << 20
+    # two heads of the Wan2.1 grid with 21248 dense rows: 166 pairs = one
+    # wave of 148 + 18 pairs cut in 8 key ranges, ~19 MB of partials
+    B, k = 1, 21248
+    need = heta.attention_workspace_size(B, 2, 128, (21, 30, 52), (3, 9, 9), k)
+    assert need > 18 << 20, need
     fake = ctypes.c_void_p(1 << 20)
-    rc = fn(fake, fake, fake, 1, 12, 128, 21, 30, 52, 3, 9, 9, ctypes.c_float(0.088), fake, k,
+    rc = fn(fake, fake, fake, B, 2, 128, 21, 30, 52, 3, 9, 9, ctypes.c_float(0.088), fake, k,
             fake, None, None)
     assert rc == heta.HETA_ERR_UNSUPPORTED

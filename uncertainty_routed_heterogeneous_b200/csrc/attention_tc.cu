@@ -73,7 +73,7 @@ struct Params {
     int Tg, Hg, Wg, wt, wh, ww;
     float scale_log2;
     // DENSE items
-    int tiles_d, pairs_d, nsplit, n_kv_d, kv_per_split, n_dense_items;
+    int tiles_d, pairs_d, pairs_full, nsplit, n_kv_d, kv_per_split, n_dense_items;
     // LOCAL items
     int box_t, box_h, box_w;
     int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
@@ -154,7 +154,8 @@ struct Item {
     int tile[2];     // query tile (DENSE) / box (LOCAL) of each slot
     int kv_lo, n;    // K/V tiles [kv_lo, kv_lo + n)
     int split;       // DENSE: which key range
-    int pair_id;     // DENSE: global pair index (for the split merge)
+    int nsplit;      // DENSE: key ranges of this pair (1: the whole range)
+    int pair_id;     // DENSE, nsplit > 1: index among the split pairs (for the merge)
     int kb;          // dense rows of sample b (n == 0: a DENSE pair past them, skipped)
 };
 
@@ -162,23 +163,36 @@ __device__ __forceinline__ Item decode(const Params &p, int id)
 {
     Item it;
     if (id < p.n_dense_items) {
-        const int per_bh = p.pairs_d * p.nsplit;
+        // the first pairs_full pairs whole, then each remaining pair in
+        // nsplit key ranges
+        int pg, kv_per;
+        if (id < p.pairs_full) {
+            pg = id;
+            it.split = 0;
+            it.nsplit = 1;
+            kv_per = p.n_kv_d;
+        } else {
+            const int r = id - p.pairs_full;
+            pg = p.pairs_full + r / p.nsplit;
+            it.split = r % p.nsplit;
+            it.nsplit = p.nsplit;
+            kv_per = p.kv_per_split;
+        }
         it.mode = DENSE;
-        it.bh = id / per_bh;
-        const int r = id % per_bh;
-        const int pair = r / p.nsplit;
-        it.split = r % p.nsplit;
-        it.pair_id = it.bh * p.pairs_d + pair;
+        it.bh = pg / p.pairs_d;
+        const int pair = pg % p.pairs_d;
+        it.pair_id = pg - p.pairs_full;
         it.tile[0] = 2 * pair;
         it.tile[1] = 2 * pair + 1;
-        it.kv_lo = it.split * p.kv_per_split;
-        it.n = min(p.n_kv_d, it.kv_lo + p.kv_per_split) - it.kv_lo;
+        it.kv_lo = it.split * kv_per;
+        it.n = min(p.n_kv_d, it.kv_lo + kv_per) - it.kv_lo;
     } else {
         const int id2 = id - p.n_dense_items;
         it.mode = LOCAL;
         it.bh = id2 / p.pairs_l;
         const int pair = id2 % p.pairs_l;
         it.split = 0;
+        it.nsplit = 1;
         it.pair_id = 0;
         it.tile[0] = 2 * pair;
         it.tile[1] = 2 * pair + 1;
@@ -782,10 +796,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 ++lc;
             }
             uint4 *dst = reinterpret_cast<uint4 *>(p.out + (row0 + token) * D);
-            if (dense && p.nsplit > 1) {
+            if (dense && it.nsplit > 1) {
                 // ---- split key range: publish this partial; the last split merges
                 const int64_t prow =
-                    ((int64_t)(it.pair_id * p.nsplit + it.split) * 2 + t) * kTileRows + r;
+                    ((int64_t)(it.pair_id * it.nsplit + it.split) * 2 + t) * kTileRows + r;
                 float4 *po = reinterpret_cast<float4 *>(p.part_o + prow * D);
 #pragma unroll
                 for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -804,19 +818,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                 if (r == 0) sh.fix_old[t] = atomicAdd(p.fix_count + it.pair_id * 2 + t, 1);
                 named_bar(1 + t, kTileRows);
                 const int old = *reinterpret_cast<volatile int *>(&sh.fix_old[t]);
-                if (old == p.nsplit - 1) {
+                if (old == it.nsplit - 1) {
                     __threadfence();
                     float mm = m_run;
-                    for (int sp = 0; sp < p.nsplit; ++sp) {
+                    for (int sp = 0; sp < it.nsplit; ++sp) {
                         if (sp == it.split) continue;
                         const int64_t orow =
-                            ((int64_t)(it.pair_id * p.nsplit + sp) * 2 + t) * kTileRows + r;
+                            ((int64_t)(it.pair_id * it.nsplit + sp) * 2 + t) * kTileRows + r;
                         mm = fmaxf(mm, __ldcg(p.part_ml + orow).x);
                     }
                     float L = 0.f;
-                    for (int sp = 0; sp < p.nsplit; ++sp) {
+                    for (int sp = 0; sp < it.nsplit; ++sp) {
                         const int64_t orow =
-                            ((int64_t)(it.pair_id * p.nsplit + sp) * 2 + t) * kTileRows + r;
+                            ((int64_t)(it.pair_id * it.nsplit + sp) * 2 + t) * kTileRows + r;
                         const float2 ml = __ldcg(p.part_ml + orow);
                         L += ml.y * ex2(ml.x - mm);
                     }
@@ -826,9 +840,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                         float acc[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-                        for (int sp = 0; sp < p.nsplit; ++sp) {
+                        for (int sp = 0; sp < it.nsplit; ++sp) {
                             const int64_t orow =
-                                ((int64_t)(it.pair_id * p.nsplit + sp) * 2 + t) * kTileRows + r;
+                                ((int64_t)(it.pair_id * it.nsplit + sp) * 2 + t) * kTileRows + r;
                             const float a = ex2(__ldcg(p.part_ml + orow).x - mm);
                             const float4 *src = reinterpret_cast<const float4 *>(p.part_o + orow * D);
                             const float4 x0 = __ldcg(src + 2 * c8), x1 = __ldcg(src + 2 * c8 + 1);
@@ -946,11 +960,24 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     pl.tiles_d = (k + kTileRows - 1) / kTileRows;
     pl.pairs_d = (pl.tiles_d + 1) / 2;
     const int64_t pairs_total = (int64_t)B * H * pl.pairs_d;
-    // split the key range in two when the dense pairs alone would not fill the SMs
-    // several times over; the LOCAL items then fill in behind the halves
-    pl.nsplit = (k > 0 && pairs_total < 4 * kPlanSMs && pl.n_kv_d >= 16) ? 2 : 1;
+    // Whole waves of pairs (a multiple of the SM count) run over the whole key
+    // range; the pairs of the last, partial wave are cut into nsplit key
+    // ranges (2..8, at least 8 tiles each) so that they spread over the SMs,
+    // and the range that finishes last merges the others' partial results.
+    // The LOCAL items fill in behind.
+    pl.pairs_full = (int)pairs_total;
+    pl.nsplit = 1;
+    if (k > 0 && pl.n_kv_d >= 16) {
+        pl.pairs_full = (int)(pairs_total / kPlanSMs * kPlanSMs);
+        const int64_t rest = pairs_total - pl.pairs_full;
+        if (rest > 0)
+            pl.nsplit = (int)max((int64_t)2, min((int64_t)min(8, pl.n_kv_d / 8), kPlanSMs / rest));
+        else
+            pl.pairs_full = (int)pairs_total;
+    }
     pl.kv_per_split = (pl.n_kv_d + pl.nsplit - 1) / pl.nsplit;
-    pl.n_dense_items = (int)(pairs_total * pl.nsplit);
+    const int64_t pairs_split = pairs_total - pl.pairs_full;
+    pl.n_dense_items = (int)(pl.pairs_full + pairs_split * pl.nsplit);
     // LOCAL query box: of the 128-token shapes below, the one whose boxes'
     // K/V covers hold the fewest keys in all (a box's cover spans the union of
     // its rows' windows, rounded up to whole 1x8x16 key sub-tiles); ties keep
@@ -988,10 +1015,10 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     pl.total_items = pl.n_dense_items + pl.n_local_items;
     // workspace: counter | split arrivals | (m,l) partials | O partials
     pl.off_fix = 256;
-    const size_t fix_bytes = pl.nsplit > 1 ? (size_t)pairs_total * 2 * sizeof(int) : 0;
+    const size_t fix_bytes = pl.nsplit > 1 ? (size_t)pairs_split * 2 * sizeof(int) : 0;
     pl.zero_bytes = pl.off_fix + fix_bytes;
     pl.off_ml = align_up(pl.zero_bytes, 256);
-    const size_t rows = pl.nsplit > 1 ? (size_t)pairs_total * pl.nsplit * 2 * kTileRows : 0;
+    const size_t rows = pl.nsplit > 1 ? (size_t)pairs_split * pl.nsplit * 2 * kTileRows : 0;
     pl.off_o = align_up(pl.off_ml + rows * sizeof(float2), 256);
     pl.workspace_bytes = pl.off_o + rows * d * sizeof(float);
     return pl;
@@ -1009,7 +1036,8 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     p.B = a.B; p.H = a.H; p.N = a.N; p.k = a.k;
     p.Tg = a.Tg; p.Hg = a.Hg; p.Wg = a.Wg; p.wt = a.wt; p.wh = a.wh; p.ww = a.ww;
     p.scale_log2 = a.scale * 1.4426950408889634f;
-    p.tiles_d = pl.tiles_d; p.pairs_d = pl.pairs_d; p.nsplit = pl.nsplit;
+    p.tiles_d = pl.tiles_d; p.pairs_d = pl.pairs_d; p.pairs_full = pl.pairs_full;
+    p.nsplit = pl.nsplit;
     p.n_kv_d = pl.n_kv_d; p.kv_per_split = pl.kv_per_split; p.n_dense_items = pl.n_dense_items;
     p.box_t = pl.box_t; p.box_h = pl.box_h; p.box_w = pl.box_w;
     p.tiles_l = pl.tiles_l; p.pairs_l = pl.pairs_l; p.nbh = pl.nbh; p.nbw = pl.nbw;

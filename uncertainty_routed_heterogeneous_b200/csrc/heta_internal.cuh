@@ -46,7 +46,7 @@ struct AttnArgs {
 
 // How one heta_attention call is cut into work items, and its workspace.
 struct AttnPlan {
-    int tiles_d, pairs_d, n_kv_d, nsplit, kv_per_split, n_dense_items;
+    int tiles_d, pairs_d, n_kv_d, pairs_full, nsplit, kv_per_split, n_dense_items;
     int box_t, box_h, box_w;  // LOCAL query box (box_t * box_h * box_w == 128)
     int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
     int total_items;
