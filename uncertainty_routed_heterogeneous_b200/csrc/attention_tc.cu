@@ -746,6 +746,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             int wbias_w0 = -(1 << 30);   // w of the first column wbias2 was built for
 #pragma unroll
             for (int c = 0; c < kKvW / 2; ++c) wbias2[c] = 0ull;
+            int jt = 0, jh = 0, jw = 0;  // LOCAL: the step's sub-tile in (t, h, w) order
             for (int j = 0; j < it.n; ++j) {
                 if (!wait(sh.s_full[t], sc & 1u)) { ok = false; break; }
                 ++sc;
@@ -759,8 +760,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                         softmax_tile<D, kPrefix>(tS, tO, j > 0, valid, wbias2, 0u, 0xFFu,
                                                  p.scale_log2, m_run, l);
                 } else {
-                    const int jt = j / (p.nkh * p.nkw), jh = (j / p.nkw) % p.nkh, jw = j % p.nkw;
                     const int kt = bx.tlo + jt, kh0 = bx.hlo + jh * kKvH, kw0 = bx.wlo + jw * kKvW;
+                    if (++jw == p.nkw) {
+                        jw = 0;
+                        if (++jh == p.nkh) {
+                            jh = 0;
+                            ++jt;
+                        }
+                    }
                     if (kw0 != wbias_w0) {
                         // columns kw0 .. kw0+15 inside the row's w-window get bias 0
                         wbias_w0 = kw0;
@@ -769,11 +776,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                             wbias2[c / 2] = f2((unsigned)(kw0 + c - qs_w) < (unsigned)p.ww ? 0u : 0xff800000u,
                                                (unsigned)(kw0 + c + 1 - qs_w) < (unsigned)p.ww ? 0u : 0xff800000u);
                     }
+                    // rows g of the sub-tile inside the row's h-window: bits
+                    // [qs_h - kh0, qs_h - kh0 + wh) clipped to [0, 8)
                     const bool t_ok = (unsigned)(kt - qs_t) < (unsigned)p.wt;
-                    uint32_t gmask = 0;
-#pragma unroll
-                    for (int g = 0; g < kKvH; ++g)
-                        gmask |= (t_ok && (unsigned)(kh0 + g - qs_h) < (unsigned)p.wh ? 1u : 0u) << g;
+                    const int glo = max(qs_h - kh0, 0), ghi = min(qs_h - kh0 + p.wh, kKvH);
+                    const uint32_t gmask =
+                        t_ok && glo < ghi ? ((1u << ghi) - 1u) & ~((1u << glo) - 1u) : 0u;
                     // groups no row of this warp sees are skipped (their P is zero)
                     const uint32_t active = __reduce_or_sync(0xffffffffu, gmask);
                     softmax_tile<D, kWindow>(tS, tO, j > 0, 0, wbias2, gmask, active,
