@@ -431,7 +431,8 @@ def run_heta(args, info):
         t_counts = torch.empty(w.B, dtype=torch.int32, device=dev)
         t_dense = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
         t_local = torch.empty((w.B, w.N), dtype=torch.int32, device=dev)
-        ws_t = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, w.N),
+        ws_t = torch.empty(heta.attention_counts_workspace_size(w.B, w.H, w.d, w.grid, w.win,
+                                                                w.N),
                            dtype=torch.uint8, device=dev)
 
         def thr_step(ev=None):

@@ -221,12 +221,23 @@ HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
  *              is not read).  heta_route_threshold writes k_cap = N rows.
  *   counts     [B] int32 (device): |D_b|; values outside 0..k_cap are
  *              clamped to it.
- *   workspace  at least heta_attention_workspace_size(..., k = k_cap) bytes.
+ *   workspace  at least heta_attention_counts_workspace_size(..., k_cap) bytes.
  *
  * Every other argument, requirement and error is as for heta_attention with
- * k = k_cap.  The work is planned for k_cap dense rows per sample; work
- * items past a sample's count end at once, so a generous k_cap costs little.
+ * k = k_cap, and B <= 1024 (else HETA_ERR_UNSUPPORTED).  The kernel cuts the
+ * dense work from the real counts, on the device, the way heta_attention
+ * cuts it from k; a generous k_cap costs only a few skipped work ids.
  */
+/*
+ * heta_attention_counts_workspace_size -- device scratch one
+ * heta_attention_counts call needs (host-only).  It covers whatever counts
+ * the device finds (at most ~20 MB at d = 128; 256 bytes when the key range
+ * is too short to split).  Same argument rules as heta_attention_counts.
+ */
+HETA_API heta_status heta_attention_counts_workspace_size(int B, int H, int d, int Tg, int Hg,
+                                                          int Wg, int wt, int wh, int ww,
+                                                          int k_cap, size_t *bytes);
+
 HETA_API heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K,
                                            const uint16_t *V, int B, int H, int d, int Tg,
                                            int Hg, int Wg, int wt, int wh, int ww, float scale,

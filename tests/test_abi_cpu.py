@@ -35,7 +35,8 @@ def test_header_declares_the_three_path_calls():
     names = declared_symbols()
     assert {"heta_route", "heta_attention", "heta_uncertainty", "heta_dense_count",
             "heta_status_string", "heta_version", "heta_attention_workspace_size",
-            "heta_route_threshold", "heta_attention_counts", "heta_route_swap"} <= names
+            "heta_route_threshold", "heta_attention_counts", "heta_route_swap",
+            "heta_attention_counts_workspace_size"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -196,3 +197,9 @@ def test_workspace_size(lib):
     assert heta.attention_workspace_size(1, 2, 64, (4, 8, 8), (3, 3, 3), 200) == 256
     with pytest.raises(heta.HetaError):
         heta.attention_workspace_size(1, 2, 96, (4, 8, 8), (3, 3, 3), 10)
+    # per-sample counts: scratch for the worst remainder the device may find,
+    # at most one wave of key ranges (148 * 2 tiles * 128 rows * 520 bytes)
+    wc = heta.attention_counts_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), 32760)
+    assert part <= wc <= 148 * 2 * 128 * (128 * 4 + 8) + 4096
+    with pytest.raises(heta.HetaError):
+        heta.attention_counts_workspace_size(1025, 1, 128, (21, 30, 52), (3, 9, 9), 100)

@@ -75,6 +75,9 @@ def load():
     lib.heta_attention_counts.argtypes = ([vp, vp, vp] + [i] * 9 +
                                           [f, vp, i, vp, vp, vp, ctypes.c_size_t, vp, vp])
     lib.heta_attention_counts.restype = i
+    lib.heta_attention_counts_workspace_size.argtypes = ([i] * 10 +
+                                                         [ctypes.POINTER(ctypes.c_size_t)])
+    lib.heta_attention_counts_workspace_size.restype = i
     _lib = lib
     return lib
 
@@ -263,6 +266,16 @@ def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=Non
     return out
 
 
+def attention_counts_workspace_size(B, H, d, grid, win, k_cap) -> int:
+    """Bytes of device scratch one ``attention_counts`` call needs."""
+    n = ctypes.c_size_t(0)
+    _check(load().heta_attention_counts_workspace_size(int(B), int(H), int(d), grid[0], grid[1],
+                                                       grid[2], win[0], win[1], win[2],
+                                                       int(k_cap), ctypes.byref(n)),
+           "heta_attention_counts_workspace_size")
+    return int(n.value)
+
+
 def attention_counts(Q, K, V, grid, win, dense_idx, counts, *, scale=None, out=None,
                      status=None, workspace=None):
     """``attention`` with per-sample dense counts on the device
@@ -289,7 +302,7 @@ def attention_counts(Q, K, V, grid, win, dense_idx, counts, *, scale=None, out=N
     po = _dev(out, torch.bfloat16, "out", 4)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    need = attention_workspace_size(B, H, d, grid, win, k_cap)
+    need = attention_counts_workspace_size(B, H, d, grid, win, k_cap)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=Q.device)
     pw = _dev(workspace, torch.uint8, "workspace", 1)

@@ -159,35 +159,81 @@ struct Item {
     int kb;          // dense rows of sample b (n == 0: a DENSE pair past them, skipped)
 };
 
-__device__ __forceinline__ Item decode(const Params &p, int id)
+// How the DENSE work is cut, worked out on the device from the real dense
+// rows (with per-sample counts only the device knows them): whole waves of
+// query-tile pairs (a multiple of the SM count) unsplit, the pairs of the last,
+// partial wave in nsplit key ranges.  Item ids [0, n_dense) are DENSE work,
+// the LOCAL items follow.
+struct DPlan {
+    int pairs_total, pairs_full, nsplit, kv_per_split, n_dense;
+};
+
+// The same rule as plan_attention's on the host.
+__device__ __forceinline__ DPlan dense_plan(int pairs_total, int n_kv)
+{
+    DPlan d;
+    d.pairs_total = pairs_total;
+    d.pairs_full = pairs_total;
+    d.nsplit = 1;
+    if (pairs_total > 0 && n_kv >= 16) {
+        d.pairs_full = pairs_total / kPlanSMs * kPlanSMs;
+        const int rest = pairs_total - d.pairs_full;
+        d.nsplit = rest > 0 ? min(min(8, n_kv / 8), kPlanSMs / rest) : 1;
+        if (d.nsplit < 2) {  // a last wave more than half full runs whole
+            d.nsplit = 1;
+            d.pairs_full = pairs_total;
+        }
+    }
+    d.kv_per_split = (n_kv + d.nsplit - 1) / d.nsplit;
+    d.n_dense = d.pairs_full + (pairs_total - d.pairs_full) * d.nsplit;
+    return d;
+}
+
+// cpref (per-sample counts only): sample b's query-tile pairs are the dense
+// pairs [H * cpref[b], H * cpref[b + 1]), ordered by head, then pair.
+__device__ __forceinline__ Item decode(const Params &p, const DPlan &dp, const int *cpref, int id)
 {
     Item it;
-    if (id < p.n_dense_items) {
+    if (id < dp.n_dense) {
         // the first pairs_full pairs whole, then each remaining pair in
         // nsplit key ranges
         int pg, kv_per;
-        if (id < p.pairs_full) {
+        if (id < dp.pairs_full) {
             pg = id;
             it.split = 0;
             it.nsplit = 1;
             kv_per = p.n_kv_d;
         } else {
-            const int r = id - p.pairs_full;
-            pg = p.pairs_full + r / p.nsplit;
-            it.split = r % p.nsplit;
-            it.nsplit = p.nsplit;
-            kv_per = p.kv_per_split;
+            const int r = id - dp.pairs_full;
+            pg = dp.pairs_full + r / dp.nsplit;
+            it.split = r % dp.nsplit;
+            it.nsplit = dp.nsplit;
+            kv_per = dp.kv_per_split;
         }
         it.mode = DENSE;
-        it.bh = pg / p.pairs_d;
-        const int pair = pg % p.pairs_d;
-        it.pair_id = pg - p.pairs_full;
+        int pair;
+        if (p.k_dev) {
+            int lo = 0, hi = p.B;  // the last b with H * cpref[b] <= pg
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (p.H * cpref[mid] <= pg) lo = mid;
+                else hi = mid;
+            }
+            const int r = pg - p.H * cpref[lo];
+            const int pairs_b = max(cpref[lo + 1] - cpref[lo], 1);
+            it.bh = lo * p.H + r / pairs_b;
+            pair = r % pairs_b;
+        } else {
+            it.bh = pg / p.pairs_d;
+            pair = pg % p.pairs_d;
+        }
+        it.pair_id = pg - dp.pairs_full;
         it.tile[0] = 2 * pair;
         it.tile[1] = 2 * pair + 1;
         it.kv_lo = it.split * kv_per;
         it.n = min(p.n_kv_d, it.kv_lo + kv_per) - it.kv_lo;
     } else {
-        const int id2 = id - p.n_dense_items;
+        const int id2 = id - dp.n_dense;
         it.mode = LOCAL;
         it.bh = id2 / p.pairs_l;
         const int pair = id2 % p.pairs_l;
@@ -347,6 +393,8 @@ struct Shared {
     int abort;
     int fix_old[2];
     uint8_t no_store[2][kTileRows];  // LOCAL: row holds a dense token
+    DPlan dplan;                     // how the DENSE work is cut (see DPlan)
+    int cpref[kMaxCountsSamples + 1];      // per-sample counts: pair prefix over samples
 };
 
 template <int D>
@@ -387,6 +435,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
         mbar_init(smem_addr(&sh.flags_empty), 2 * kTileRows);
         mbar_init(smem_addr(&sh.drain), 1);
         sh.abort = 0;
+        int pairs_total = p.B * p.H * p.pairs_d;
+        if (p.k_dev) {
+            int acc = 0;
+            for (int b = 0; b < p.B; ++b) {
+                sh.cpref[b] = acc;
+                const int kb = min(max(__ldg(p.k_dev + b), 0), p.k);
+                acc += (kb + 2 * kTileRows - 1) / (2 * kTileRows);
+            }
+            sh.cpref[p.B] = acc;
+            pairs_total = p.H * acc;
+        }
+        sh.dplan = dense_plan(pairs_total, p.n_kv_d);
         fence_mbar_init();
         fence_proxy_async_smem();
     }
@@ -398,6 +458,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sh.tmem_base;
+    const DPlan dplan = sh.dplan;
     const volatile int *abort = &sh.abort;
 
     auto fail = [&]() {
@@ -432,10 +493,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             prefetch_tmap(&tmQ5);
             uint32_t issued = 0, qi = 0, items = 0;
             bool ok = true;
-            int id = atomicAdd(p.counter, 1);
+            // the next item id; -1 when none is left
+            const int total_items = dplan.n_dense + p.n_local_items;
+            auto grab = [&]() -> int {
+                const int g = atomicAdd(p.counter, 1);
+                return g < total_items ? g : -1;
+            };
+            int id = grab();
             while (ok) {
-                if (id >= p.total_items) id = -1;
-                const int next = id >= 0 ? atomicAdd(p.counter, 1) : -1;
+                const int next = id >= 0 ? grab() : -1;
                 // publish the item
                 {
                     const int slot = qi % kQueue;
@@ -445,7 +511,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                     ++qi;
                 }
                 if (id < 0) break;
-                const Item it = decode(p, id);
+                const Item it = decode(p, dplan, sh.cpref, id);
                 if (it.n == 0) {  // a DENSE pair past the sample's dense rows: every role skips it
                     id = next;
                     continue;
@@ -555,7 +621,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             while (ok) {
                 const int id = pop_item(qi++, ok);
                 if (!ok || id < 0) break;
-                const Item it = decode(p, id);
+                const Item it = decode(p, dplan, sh.cpref, id);
                 const int n = it.n;
                 if (n == 0) continue;
                 const bool dense = it.mode == DENSE;
@@ -639,7 +705,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
         while (ok) {
             const int id = pop_item(qi++, ok);
             if (!ok || id < 0) break;
-            const Item it = decode(p, id);
+            const Item it = decode(p, dplan, sh.cpref, id);
             if (it.mode != LOCAL) continue;
             if (!wait(sh.flags_empty, (lc & 1u) ^ 1u)) { ok = false; break; }
             for (int t = 0; t < 2; ++t)
@@ -705,7 +771,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
         while (ok) {
             const int id = pop_item(qi++, ok);
             if (!ok || id < 0) break;
-            const Item it = decode(p, id);
+            const Item it = decode(p, dplan, sh.cpref, id);
             if (it.n == 0) continue;
             const bool dense = it.mode == DENSE;
             const int tile = it.tile[t];
@@ -970,22 +1036,43 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     const int64_t pairs_total = (int64_t)B * H * pl.pairs_d;
     // Whole waves of pairs (a multiple of the SM count) run over the whole key
     // range; the pairs of the last, partial wave are cut into nsplit key
-    // ranges (2..8, at least 8 tiles each) so that they spread over the SMs,
-    // and the range that finishes last merges the others' partial results.
+    // ranges (2..8, at least 8 tiles each, at most one wave of ranges) so that
+    // they spread over the SMs, and the range that finishes last merges the
+    // others' partial results; a last wave more than half full runs whole.
     // The LOCAL items fill in behind.
     pl.pairs_full = (int)pairs_total;
     pl.nsplit = 1;
     if (k > 0 && pl.n_kv_d >= 16) {
         pl.pairs_full = (int)(pairs_total / kPlanSMs * kPlanSMs);
         const int64_t rest = pairs_total - pl.pairs_full;
-        if (rest > 0)
-            pl.nsplit = (int)max((int64_t)2, min((int64_t)min(8, pl.n_kv_d / 8), kPlanSMs / rest));
-        else
+        pl.nsplit = rest > 0 ? (int)min((int64_t)min(8, pl.n_kv_d / 8), kPlanSMs / rest) : 1;
+        if (pl.nsplit < 2) {  // a last wave more than half full runs whole
+            pl.nsplit = 1;
             pl.pairs_full = (int)pairs_total;
+        }
     }
     pl.kv_per_split = (pl.n_kv_d + pl.nsplit - 1) / pl.nsplit;
-    const int64_t pairs_split = pairs_total - pl.pairs_full;
-    pl.n_dense_items = (int)(pl.pairs_full + pairs_split * pl.nsplit);
+    int64_t pairs_split = pairs_total - pl.pairs_full;  // pairs cut into key ranges
+    int64_t split_ranges = pairs_split * pl.nsplit;      // their ranges
+    pl.n_dense_items = (int)(pl.pairs_full + split_ranges);
+    if (per_sample_counts) {
+        // The device plans from the real counts (at most k per sample), the
+        // same way: reserve ids and scratch for the worst remainder.
+        int64_t extra = 0, worst_split = 0, worst_ranges = 0;
+        if (k > 0 && pl.n_kv_d >= 16) {
+            for (int rest = 1; rest < kPlanSMs && rest <= pairs_total; ++rest) {
+                const int ns = min(min(8, pl.n_kv_d / 8), kPlanSMs / rest);
+                if (ns < 2) continue;
+                extra = max(extra, (int64_t)rest * (ns - 1));
+                worst_split = rest;
+                worst_ranges = max(worst_ranges, (int64_t)rest * ns);
+            }
+        }
+        pl.n_dense_items = (int)(pairs_total + extra);
+        pairs_split = worst_split;
+        split_ranges = worst_ranges;
+        pl.nsplit = max(pl.nsplit, 2);  // (the scratch below is sized by the ranges)
+    }
     // LOCAL query box: of the 128-token shapes below, the one whose boxes'
     // K/V covers hold the fewest keys in all (a box's cover spans the union of
     // its rows' windows, rounded up to whole 1x8x16 key sub-tiles); ties keep
@@ -1023,10 +1110,10 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     pl.total_items = pl.n_dense_items + pl.n_local_items;
     // workspace: counter | split arrivals | (m,l) partials | O partials
     pl.off_fix = 256;
-    const size_t fix_bytes = pl.nsplit > 1 ? (size_t)pairs_split * 2 * sizeof(int) : 0;
+    const size_t fix_bytes = split_ranges > 0 ? (size_t)pairs_split * 2 * sizeof(int) : 0;
     pl.zero_bytes = pl.off_fix + fix_bytes;
     pl.off_ml = align_up(pl.zero_bytes, 256);
-    const size_t rows = pl.nsplit > 1 ? (size_t)pairs_split * pl.nsplit * 2 * kTileRows : 0;
+    const size_t rows = split_ranges > 0 ? (size_t)split_ranges * 2 * kTileRows : 0;
     pl.off_o = align_up(pl.off_ml + rows * sizeof(float2), 256);
     pl.workspace_bytes = pl.off_o + rows * d * sizeof(float);
     return pl;

@@ -127,6 +127,19 @@ heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg, i
     return HETA_OK;
 }
 
+heta_status heta_attention_counts_workspace_size(int B, int H, int d, int Tg, int Hg, int Wg,
+                                                 int wt, int wh, int ww, int k_cap,
+                                                 size_t *bytes)
+{
+    if (!bytes) return HETA_ERR_INVALID_ARG;
+    const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k_cap);
+    if (st != HETA_OK) return st;
+    if (B > heta::kMaxCountsSamples) return HETA_ERR_UNSUPPORTED;
+    *bytes = heta::plan_attention(B, H, d, Tg * Hg * Wg, k_cap, Tg, Hg, Wg, wt, wh, ww, true)
+                 .workspace_bytes;
+    return HETA_OK;
+}
+
 heta_status heta_attention(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B,
                            int H, int d, int Tg, int Hg, int Wg, int wt, int wh, int ww,
                            float scale, const int32_t *dense_idx, int k, uint16_t *out,
@@ -161,6 +174,7 @@ heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K, const ui
 {
     const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k_cap);
     if (st != HETA_OK) return st;
+    if (B > heta::kMaxCountsSamples) return HETA_ERR_UNSUPPORTED;
     const int N = Tg * Hg * Wg;
     if (!(scale > 0.f) || !isfinite(scale)) return HETA_ERR_INVALID_ARG;
     if (!Q || !K || !V || !out || !counts || (k_cap > 0 && !dense_idx) || !workspace)

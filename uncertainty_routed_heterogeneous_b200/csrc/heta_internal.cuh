@@ -57,6 +57,10 @@ struct AttnPlan {
 // on it, never the result; the launch itself uses the device's real count.
 constexpr int kPlanSMs = 148;
 
+// Samples heta_attention_counts takes (its per-sample pair prefix lives in
+// shared memory).
+constexpr int kMaxCountsSamples = 1024;
+
 // k is the dense rows per sample, or their capacity when per_sample_counts
 // (the counts are then only known on the device: LOCAL items are always planned).
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
