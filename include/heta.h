@@ -162,11 +162,12 @@ HETA_API heta_status heta_route_threshold(const float *u, int B, int N, double c
  * needs for these sizes (host-only; touches no device).
  *
  * The scratch holds the work-item counter of the persistent kernel and, when
- * the pairs of dense query tiles of the last, partial wave of work are cut
- * into 2..8 key ranges to keep all SMs busy, the partial results those
- * ranges merge (fp32, about 1 KB per row and range, half for d = 64; at most
- * ~19 MB).  At the Wan2.1-1.3B shape with rho = 0.2 that is about 17 MB;
- * when the dense pairs make whole waves it is 256 bytes.  Same argument rules as
+ * the pairs of dense query tiles of a last, at most half-full wave of work
+ * (or of a first and only, partial one) are cut into two key ranges to keep
+ * all SMs busy, the partial results those ranges merge (fp32, about 1 KB per
+ * row and range, half for d = 64; at most ~40 MB).  At the Wan2.1-1.3B
+ * shape that is about 4 MB for rho = 0.2 and 22 MB for rho = 0.05; when no
+ * pair is cut it is 256 bytes.  Same argument rules as
  * heta_attention; *bytes is only written on HETA_OK.
  */
 HETA_API heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg,
@@ -231,7 +232,7 @@ HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
 /*
  * heta_attention_counts_workspace_size -- device scratch one
  * heta_attention_counts call needs (host-only).  It covers whatever counts
- * the device finds (at most ~20 MB at d = 128; 256 bytes when the key range
+ * the device finds (at most ~40 MB at d = 128; 256 bytes when the key range
  * is too short to split).  Same argument rules as heta_attention_counts.
  */
 HETA_API heta_status heta_attention_counts_workspace_size(int B, int H, int d, int Tg, int Hg,
@@ -257,10 +258,11 @@ HETA_API heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K,
  * except the workspace, and allocates nothing.
  *
  * Its scratch is a fixed 16 MiB array in the library's device memory, which
- * every GPU that loads the library keeps until the process exits.  Sizes
- * whose scratch (heta_attention_workspace_size) exceeds 16 MiB are rejected
- * with HETA_ERR_UNSUPPORTED before anything is launched; use heta_attention
- * for those.  The first call on each device looks up the array's device
+ * every GPU that loads the library keeps until the process exits.  When
+ * the scratch heta_attention would use (heta_attention_workspace_size)
+ * exceeds 16 MiB, no dense pair is cut into key ranges: the kernel then needs
+ * only its work counter, and the result is the same up to rounding order
+ * (a partly filled last wave of dense work takes longer).  The first call on each device looks up the array's device
  * address (a host-side runtime query, done once per device with that device
  * current), so make the first call on a device before any stream capture.
  * All calls share the array and it keeps the last call's contents; each call

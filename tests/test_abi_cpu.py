@@ -181,13 +181,21 @@ def test_flop_model_matches_the_papers_reduction():
 
 def test_workspace_size(lib):
     """Whole waves of dense pairs run unsplit and need no scratch beyond the
-    work counter; the pairs of the last, partial wave are cut into 2..8 key
-    ranges whose fp32 partials the workspace holds."""
-    # rho = 0.2: 312 pairs = 2 waves of 148 + 16 pairs cut in 8 (148 // 16 = 9 -> 8)
+    work counter; the pairs of a last wave at most half full (or of a first
+    and only, partial wave) are cut into two key ranges whose fp32 partials
+    the workspace holds."""
+    # rho = 0.2: 312 pairs = 2 waves of 148 + 16 pairs cut in halves
     k = heta.dense_count(32760, 0.2)
     part = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k)
-    assert part >= 16 * 8 * 2 * 128 * (128 * 4 + 8)
-    assert part < 20 * 2 ** 20
+    assert part >= 16 * 2 * 2 * 128 * (128 * 4 + 8)
+    assert part < 5 * 2 ** 20
+    # a last wave more than half full runs whole: counter only
+    k_full = heta.dense_count(32760, 0.15)  # 240 pairs = 148 + 92
+    assert heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k_full) == 256
+    # one partial wave (rho = 0.05: 84 pairs) is cut in halves as well
+    k_small = heta.dense_count(32760, 0.05)
+    w_small = heta.attention_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), k_small)
+    assert w_small >= 84 * 2 * 2 * 128 * (128 * 4 + 8)
     # exactly whole waves: 148 pairs of 2 tiles -> no split, counter only
     k148 = 148 * 256
     w = heta.attention_workspace_size(1, 1, 128, (37, 32, 32), (3, 9, 9), k148)
@@ -198,8 +206,9 @@ def test_workspace_size(lib):
     with pytest.raises(heta.HetaError):
         heta.attention_workspace_size(1, 2, 96, (4, 8, 8), (3, 3, 3), 10)
     # per-sample counts: scratch for the worst remainder the device may find,
-    # at most one wave of key ranges (148 * 2 tiles * 128 rows * 520 bytes)
+    # at most 147 pairs in halves (147 * 2 ranges * 2 tiles * 128 rows * 520 bytes)
     wc = heta.attention_counts_workspace_size(1, 12, 128, (21, 30, 52), (3, 9, 9), 32760)
-    assert part <= wc <= 148 * 2 * 128 * (128 * 4 + 8) + 4096
+    assert max(part, w_small) <= wc <= 147 * 2 * 2 * 128 * (128 * 4 + 8) + 4096
+    assert wc > 32 << 20
     with pytest.raises(heta.HetaError):
         heta.attention_counts_workspace_size(1025, 1, 128, (21, 30, 52), (3, 9, 9), 100)

@@ -5,8 +5,8 @@ run), so they cannot hand heta_attention a workspace.  heta_attention_noalloc
 takes the same arguments minus the workspace and keeps its scratch in a fixed
 16 MiB array inside the library.  This file checks, through the C ABI, that
 its output matches heta_attention's on two calls in a row (the second call
-reuses the array the first one left behind), and that sizes whose scratch
-would not fit are refused before anything runs.
+reuses the array the first one left behind), and that a size whose split
+scratch would not fit runs unsplit with the same result.
 
 The file name sorts last so that a run stopping at the first failure has run
 every other test first.
@@ -66,17 +66,34 @@ def test_noalloc_matches_workspace_entry_point(gpu_lib, grid, win, rho, H, d):
         assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (call, err.max(), err.mean())
 
 
-def test_noalloc_refuses_sizes_beyond_its_array(gpu_lib):
-    """A call whose scratch would not fit the 16 MiB array is refused up front,
-    before anything is launched (the pointers below are never touched)."""
+def test_noalloc_runs_unsplit_when_its_array_is_too_small(gpu_lib):
+    """A size whose split partials would not fit the 16 MiB array runs with
+    every dense pair over its whole key range and still matches
+    heta_attention (which splits)."""
+    import torch
     heta = gpu_lib
     fn = _noalloc(heta.load())
-    # two heads of the Wan2.1 grid with 21248 dense rows: 166 pairs = one
-    # wave of 148 + 18 pairs cut in 8 key ranges, ~19 MB of partials
-    B, k = 1, 21248
-    need = heta.attention_workspace_size(B, 2, 128, (21, 30, 52), (3, 9, 9), k)
-    assert need > 18 << 20, need
-    fake = ctypes.c_void_p(1 << 20)
-    rc = fn(fake, fake, fake, B, 2, 128, 21, 30, 52, 3, 9, 9, ctypes.c_float(0.088), fake, k,
-            fake, None, None)
-    assert rc == heta.HETA_ERR_UNSUPPORTED
+    # two heads of the Wan2.1 grid with 28416 dense rows: 222 pairs = one
+    # wave of 148 + 74 pairs cut in halves, ~19.5 MB of partials
+    grid, win, kk = (21, 30, 52), (3, 9, 9), 28416
+    assert heta.attention_workspace_size(1, 2, 128, grid, win, kk) > 16 << 20
+    w = W.scaled(W.WAN21, H=2, d=128, grid=grid, win=win, u_kind="uniform", u_seeds=(5,))
+    q, k, v = W.make_qkv(w)
+    Q, K, V = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+    dense, _, _, _ = heta.route(to_dev(W.make_u(w)), kk)
+    want = from_dev_bf16(heta.attention(Q, K, V, grid, win, dense))
+    out = torch.full_like(Q, float("nan"))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = fn(ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(K.data_ptr()),
+            ctypes.c_void_p(V.data_ptr()), 1, 2, 128, grid[0], grid[1], grid[2],
+            win[0], win[1], win[2], ctypes.c_float(1.0 / math.sqrt(128)),
+            ctypes.c_void_p(dense.data_ptr()), kk, ctypes.c_void_p(out.data_ptr()),
+            ctypes.c_void_p(st.data_ptr()), stream)
+    assert rc == heta.HETA_OK, heta.status_string(rc)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    got = from_dev_bf16(out)
+    assert np.all(np.isfinite(got))
+    err = np.abs(got - want)
+    assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())

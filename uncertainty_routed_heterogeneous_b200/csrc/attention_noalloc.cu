@@ -2,7 +2,7 @@
 //
 // heta_attention needs device scratch (the work-item counter of the
 // persistent kernel and, when the dense rows' key range is split, the halves'
-// partial results).  Some callers cannot provide it: code that must not call
+// partial results; without the split only the counter).  Some callers cannot provide it: code that must not call
 // cudaMalloc at all (a real-time loop that may not block on the allocator, a
 // plug-in host that owns every allocation, code running where the allocator
 // is off limits).  heta_attention_noalloc runs the same kernel with its
@@ -63,11 +63,15 @@ HETA_API heta_status heta_attention_noalloc(const uint16_t *Q, const uint16_t *K
     heta_status st =
         heta_attention_workspace_size(B, H, d, Tg, Hg, Wg, wt, wh, ww, k, &need);
     if (st != HETA_OK) return st;
-    if (need > heta::kStaticScratchBytes) return HETA_ERR_UNSUPPORTED;
+    // When the halves' partials of a split last wave do not fit the array,
+    // every dense pair runs over its whole key range instead (the counter
+    // alone): slower for that wave, the same result up to rounding order.
+    const bool allow_split = need <= heta::kStaticScratchBytes;
     void *scratch = nullptr;
     if (heta::scratch_on_current_device(&scratch) != cudaSuccess) return HETA_ERR_CUDA;
-    return heta_attention(Q, K, V, B, H, d, Tg, Hg, Wg, wt, wh, ww, scale, dense_idx, k, out,
-                          scratch, heta::kStaticScratchBytes, status_dev, stream);
+    return static_cast<heta_status>(heta::attention_checked(
+        Q, K, V, B, H, d, Tg, Hg, Wg, wt, wh, ww, scale, dense_idx, k, out, scratch,
+        heta::kStaticScratchBytes, status_dev, stream, allow_split));
 }
 
 }  // extern "C"

@@ -50,6 +50,7 @@ constexpr int kRingBytes = 128 * 1024;  // K/V ring
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr float kRescaleLog2 = 8.0f;    // rescale O only when the max grows > 2^8
 constexpr int kQueue = 4;               // work-item queue depth
+constexpr int kMaxSplit = 2;            // key ranges a DENSE pair is cut into at most
 
 // query box (LOCAL) and key sub-tile
 // (the query box is planned per call among shapes of 128 tokens, see
@@ -74,6 +75,7 @@ struct Params {
     float scale_log2;
     // DENSE items
     int tiles_d, pairs_d, pairs_full, nsplit, n_kv_d, kv_per_split, n_dense_items;
+    int max_split;    // 1: no pair is cut into key ranges (the scratch has no room)
     // LOCAL items
     int box_t, box_h, box_w;
     int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
@@ -169,7 +171,7 @@ struct DPlan {
 };
 
 // The same rule as plan_attention's on the host.
-__device__ __forceinline__ DPlan dense_plan(int pairs_total, int n_kv)
+__device__ __forceinline__ DPlan dense_plan(int pairs_total, int n_kv, int max_split)
 {
     DPlan d;
     d.pairs_total = pairs_total;
@@ -178,7 +180,8 @@ __device__ __forceinline__ DPlan dense_plan(int pairs_total, int n_kv)
     if (pairs_total > 0 && n_kv >= 16) {
         d.pairs_full = pairs_total / kPlanSMs * kPlanSMs;
         const int rest = pairs_total - d.pairs_full;
-        d.nsplit = rest > 0 ? min(min(8, n_kv / 8), kPlanSMs / rest) : 1;
+        d.nsplit = rest > 0 ? min(max_split, n_kv / 8) : 1;
+        if (d.pairs_full > 0 && rest > kPlanSMs / 2) d.nsplit = 1;
         if (d.nsplit < 2) {  // a last wave more than half full runs whole
             d.nsplit = 1;
             d.pairs_full = pairs_total;
@@ -446,7 +449,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             sh.cpref[p.B] = acc;
             pairs_total = p.H * acc;
         }
-        sh.dplan = dense_plan(pairs_total, p.n_kv_d);
+        sh.dplan = dense_plan(pairs_total, p.n_kv_d, p.max_split);
         fence_mbar_init();
         fence_proxy_async_smem();
     }
@@ -1027,25 +1030,28 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 }  // namespace
 
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
-                        int wh, int ww, bool per_sample_counts)
+                        int wh, int ww, bool per_sample_counts, bool allow_split)
 {
     AttnPlan pl;
+    pl.max_split = allow_split ? kMaxSplit : 1;
     pl.n_kv_d = (N + kTileKeys - 1) / kTileKeys;
     pl.tiles_d = (k + kTileRows - 1) / kTileRows;
     pl.pairs_d = (pl.tiles_d + 1) / 2;
     const int64_t pairs_total = (int64_t)B * H * pl.pairs_d;
     // Whole waves of pairs (a multiple of the SM count) run over the whole key
-    // range; the pairs of the last, partial wave are cut into nsplit key
-    // ranges (2..8, at least 8 tiles each, at most one wave of ranges) so that
-    // they spread over the SMs, and the range that finishes last merges the
-    // others' partial results; a last wave more than half full runs whole.
-    // The LOCAL items fill in behind.
+    // range; the pairs of a last wave at most half full (or of a first and
+    // only, partial wave) are cut into two key ranges so that they spread over
+    // the SMs, and the range that finishes second merges the other's partial
+    // result; a fuller last wave runs whole.
+    // The LOCAL items fill in behind.  (Cutting into up to 8 ranges was
+    // measured slower: each merge costs more than the finer spread gains.)
     pl.pairs_full = (int)pairs_total;
     pl.nsplit = 1;
     if (k > 0 && pl.n_kv_d >= 16) {
         pl.pairs_full = (int)(pairs_total / kPlanSMs * kPlanSMs);
         const int64_t rest = pairs_total - pl.pairs_full;
-        pl.nsplit = rest > 0 ? (int)min((int64_t)min(8, pl.n_kv_d / 8), kPlanSMs / rest) : 1;
+        pl.nsplit = rest > 0 ? min(pl.max_split, pl.n_kv_d / 8) : 1;
+        if (pl.pairs_full > 0 && rest > kPlanSMs / 2) pl.nsplit = 1;
         if (pl.nsplit < 2) {  // a last wave more than half full runs whole
             pl.nsplit = 1;
             pl.pairs_full = (int)pairs_total;
@@ -1061,7 +1067,8 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
         int64_t extra = 0, worst_split = 0, worst_ranges = 0;
         if (k > 0 && pl.n_kv_d >= 16) {
             for (int rest = 1; rest < kPlanSMs && rest <= pairs_total; ++rest) {
-                const int ns = min(min(8, pl.n_kv_d / 8), kPlanSMs / rest);
+                // (the device's pairs_full may be 0, when the counts are small)
+                const int ns = min(pl.max_split, pl.n_kv_d / 8);
                 if (ns < 2) continue;
                 extra = max(extra, (int64_t)rest * (ns - 1));
                 worst_split = rest;
@@ -1071,7 +1078,7 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
         pl.n_dense_items = (int)(pairs_total + extra);
         pairs_split = worst_split;
         split_ranges = worst_ranges;
-        pl.nsplit = max(pl.nsplit, 2);  // (the scratch below is sized by the ranges)
+        if (worst_ranges > 0) pl.nsplit = 2;  // (the scratch below is sized by the ranges)
     }
     // LOCAL query box: of the 128-token shapes below, the one whose boxes'
     // K/V covers hold the fewest keys in all (a box's cover spans the union of
@@ -1133,6 +1140,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.tiles_d = pl.tiles_d; p.pairs_d = pl.pairs_d; p.pairs_full = pl.pairs_full;
     p.nsplit = pl.nsplit;
+    p.max_split = pl.max_split;
     p.n_kv_d = pl.n_kv_d; p.kv_per_split = pl.kv_per_split; p.n_dense_items = pl.n_dense_items;
     p.box_t = pl.box_t; p.box_h = pl.box_h; p.box_w = pl.box_w;
     p.tiles_l = pl.tiles_l; p.pairs_l = pl.pairs_l; p.nbh = pl.nbh; p.nbw = pl.nbw;

@@ -114,6 +114,35 @@ heta_status check_attention_shape(int B, int H, int d, int Tg, int Hg, int Wg, i
 
 }  // namespace
 
+namespace heta {
+
+int attention_checked(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H,
+                      int d, int Tg, int Hg, int Wg, int wt, int wh, int ww, float scale,
+                      const int32_t *dense_idx, int k, uint16_t *out, void *workspace,
+                      size_t workspace_bytes, int32_t *status_dev, void *stream,
+                      bool allow_split)
+{
+    const int N = Tg * Hg * Wg;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return HETA_ERR_INVALID_ARG;
+    if (!Q || !K || !V || !out || (k > 0 && !dense_idx) || !workspace)
+        return HETA_ERR_INVALID_ARG;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
+        (dense_idx && !aligned16(dense_idx)) || !aligned16(workspace))
+        return HETA_ERR_INVALID_ARG;
+    const AttnPlan plan =
+        plan_attention(B, H, d, N, k, Tg, Hg, Wg, wt, wh, ww, false, allow_split);
+    if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
+    AttnArgs a;
+    a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
+    a.k_dev = nullptr;
+    a.B = B; a.H = H; a.d = d; a.N = N; a.k = k;
+    a.Tg = Tg; a.Hg = Hg; a.Wg = Wg; a.wt = wt; a.wh = wh; a.ww = ww;
+    a.scale = scale;
+    return from_cuda(launch_attention(a, plan, workspace, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace heta
+
 extern "C" {
 
 heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg, int Wg, int wt,
@@ -148,22 +177,9 @@ heta_status heta_attention(const uint16_t *Q, const uint16_t *K, const uint16_t 
 {
     const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k);
     if (st != HETA_OK) return st;
-    const int N = Tg * Hg * Wg;
-    if (!(scale > 0.f) || !isfinite(scale)) return HETA_ERR_INVALID_ARG;
-    if (!Q || !K || !V || !out || (k > 0 && !dense_idx) || !workspace)
-        return HETA_ERR_INVALID_ARG;
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) ||
-        (dense_idx && !aligned16(dense_idx)) || !aligned16(workspace))
-        return HETA_ERR_INVALID_ARG;
-    const heta::AttnPlan plan = heta::plan_attention(B, H, d, N, k, Tg, Hg, Wg, wt, wh, ww);
-    if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
-    heta::AttnArgs a;
-    a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
-    a.k_dev = nullptr;
-    a.B = B; a.H = H; a.d = d; a.N = N; a.k = k;
-    a.Tg = Tg; a.Hg = Hg; a.Wg = Wg; a.wt = wt; a.wh = wh; a.ww = ww;
-    a.scale = scale;
-    return from_cuda(heta::launch_attention(a, plan, workspace, static_cast<cudaStream_t>(stream)));
+    return static_cast<heta_status>(heta::attention_checked(
+        Q, K, V, B, H, d, Tg, Hg, Wg, wt, wh, ww, scale, dense_idx, k, out, workspace,
+        workspace_bytes, status_dev, stream, true));
 }
 
 heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K, const uint16_t *V,

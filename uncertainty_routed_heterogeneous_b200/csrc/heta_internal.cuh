@@ -47,6 +47,7 @@ struct AttnArgs {
 // How one heta_attention call is cut into work items, and its workspace.
 struct AttnPlan {
     int tiles_d, pairs_d, n_kv_d, pairs_full, nsplit, kv_per_split, n_dense_items;
+    int max_split;            // most key ranges a dense pair may be cut into
     int box_t, box_h, box_w;  // LOCAL query box (box_t * box_h * box_w == 128)
     int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
     int total_items;
@@ -63,8 +64,20 @@ constexpr int kMaxCountsSamples = 1024;
 
 // k is the dense rows per sample, or their capacity when per_sample_counts
 // (the counts are then only known on the device: LOCAL items are always planned).
+// allow_split = false runs every dense pair over its whole key range, so the
+// workspace is only the work counter.
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
-                        int wh, int ww, bool per_sample_counts = false);
+                        int wh, int ww, bool per_sample_counts = false,
+                        bool allow_split = true);
+
+// heta_attention's body once its shape is checked, with the split choice open
+// (the allocation-free entry point turns splitting off when its fixed scratch
+// is too small for it).
+int attention_checked(const uint16_t *Q, const uint16_t *K, const uint16_t *V, int B, int H,
+                      int d, int Tg, int Hg, int Wg, int wt, int wh, int ww, float scale,
+                      const int32_t *dense_idx, int k, uint16_t *out, void *workspace,
+                      size_t workspace_bytes, int32_t *status_dev, void *stream,
+                      bool allow_split);
 
 cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &plan, void *workspace,
                              cudaStream_t s);
