@@ -119,9 +119,11 @@ cudaError_t launch_uncertainty(const uint16_t *X, const float *w, float bias,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    // 4 CTAs of 16 warps per SM; each warp walks rows with a grid stride
+    // One wave: the two CTAs of 16 warps an SM holds (64 registers a thread),
+    // each warp walking rows with a grid stride, so the rows split over all
+    // warps at once (a second wave would run on a partly idle GPU)
     int64_t blocks = (rows + kWarps - 1) / kWarps;
-    if (blocks > 4LL * sms) blocks = 4LL * sms;
+    if (blocks > 2LL * sms) blocks = 2LL * sms;
     uncertainty_kernel<6><<<(unsigned)blocks, kThreads, smem, s>>>(X, w, bias, rows, C, u);
     return cudaGetLastError();
 }
