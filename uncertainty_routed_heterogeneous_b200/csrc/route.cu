@@ -207,6 +207,59 @@ __device__ __forceinline__ void compact(const uint32_t *slot, int off, int t_lo,
     if (base < t_hi) step(base + lane, base + lane < t_hi);
 }
 
+// The common case of compact (float select, no token equal to T in this warp,
+// no mask) with each whole 32-token step written out as one PTX sequence:
+// load, compare, ballot, rank, one store into the list that holds the token.
+__device__ __forceinline__ void compact_float_plain(const uint32_t *slot, int off, int t_lo,
+                                                    int t_hi, uint32_t kst, uint32_t rd,
+                                                    int32_t *dout, int32_t *lout, int lane)
+{
+    const unsigned lt = (1u << lane) - 1u;
+    const int full_end = t_lo + ((t_hi - t_lo) & ~31);
+    uint32_t t = (uint32_t)(t_lo + lane);
+    uint32_t at = (uint32_t)__cvta_generic_to_shared(slot + off + t_lo + lane);
+    const uint64_t dbase = reinterpret_cast<uint64_t>(dout);
+    const uint64_t lbase = reinterpret_cast<uint64_t>(lout);
+#pragma unroll 4
+    for (int base = t_lo; base < full_end; base += 32) {
+        asm volatile(
+            "{\n\t"
+            ".reg .pred p;\n\t"
+            ".reg .b32 w, dm, c, pos, idx;\n\t"
+            ".reg .b64 lst, ptr;\n\t"
+            "ld.shared.b32 w, [%1];\n\t"
+            "setp.gt.f32 p, w, %3;\n\t"
+            "vote.sync.ballot.b32 dm, p, 0xffffffff;\n\t"
+            "and.b32 c, dm, %4;\n\t"
+            "popc.b32 c, c;\n\t"
+            "add.u32 pos, %2, c;\n\t"
+            "sub.u32 idx, %0, pos;\n\t"
+            "selp.b32 idx, pos, idx, p;\n\t"
+            "selp.b64 lst, %5, %6, p;\n\t"
+            "mad.wide.u32 ptr, idx, 4, lst;\n\t"
+            "st.global.b32 [ptr], %0;\n\t"
+            "popc.b32 c, dm;\n\t"
+            "add.u32 %2, %2, c;\n\t"
+            "add.u32 %0, %0, 32;\n\t"
+            "add.u32 %1, %1, 128;\n\t"
+            "}"
+            : "+r"(t), "+r"(at), "+r"(rd)
+            : "f"(__uint_as_float(kst)), "r"(lt), "l"(dbase), "l"(lbase)
+            : "memory");
+    }
+    if (full_end < t_hi) {  // the last, partial step
+        const bool valid = (int)t < t_hi;
+        const uint32_t w = valid ? slot[t + off] : 0u;
+        const bool dense = valid && __uint_as_float(w) > __uint_as_float(kst);
+        const unsigned dm = __ballot_sync(kFull, dense);
+        const uint32_t pos = rd + __popc(dm & lt);
+        if (valid) {
+            int32_t *const dst = dense ? dout + pos : lout + (t - pos);
+            *dst = (int32_t)t;
+        }
+    }
+}
+
 template <bool kMask>
 __global__ void __launch_bounds__(kThreads, 1)
 route_kernel(const float *__restrict__ u, int B, int N, int k,
@@ -590,9 +643,11 @@ route_kernel(const float *__restrict__ u, int B, int N, int k,
                 if (has_eq)
                     compact<false, true, kMask>(slot, off, t_lo, t_hi, kst, take, rd, re, dout,
                                                 lout, mout, ku, nl, lane);
+                else if (!kMask)
+                    compact_float_plain(slot, off, t_lo, t_hi, kst, rd, dout, lout, lane);
                 else
-                    compact<false, false, kMask>(slot, off, t_lo, t_hi, kst, take, rd, re,
-                                                 dout, lout, mout, ku, nl, lane);
+                    compact<false, false, true>(slot, off, t_lo, t_hi, kst, take, rd, re,
+                                                dout, lout, mout, ku, nl, lane);
             }
         }
         __syncthreads();  // shared memory is reused by the next sample
