@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-dense-compare", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-other-configs", action="store_true",
+                   help="skip timing the Wan2.2 shape, the batched step with the head and "
+                        "the rho sweep (uniform / clustered u)")
     p.add_argument("--no-window-sweep", action="store_true",
                    help="skip timing the 9^3 / 11^3 / 13^3 windows of the paper's ablation")
     p.add_argument("--no-threshold-mode", action="store_true",
@@ -288,6 +291,76 @@ def config_of(w, n_gpus):
 # ----------------------------------------------------------------------------
 
 
+def _time_ms(torch, fn, reps=5):
+    fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
+    """The Wan2.2-5B shape, the batched two-sample step with the head, and the
+    rho sweep on uniform and clustered u at the Wan2.1 shape: CUDA-event times
+    of the same calls as the main step (Q/K/V/X iid N(0,1) bf16 drawn on the
+    device from a seeded generator; u from the workload's own generator)."""
+    res = {}
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+
+    def randn_bf16(*shape):
+        return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+
+    def one_step(w, Q, K, V, X, wv, u):
+        kk = heta.dense_count(w.N, w.rho)
+        dense = torch.empty((w.B, kk), dtype=torch.int32, device=dev)
+        local = torch.empty((w.B, w.N - kk), dtype=torch.int32, device=dev)
+        o = torch.empty_like(Q)
+        ws = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, kk),
+                         dtype=torch.uint8, device=dev)
+        u_next = torch.empty((w.B, w.N), dtype=torch.float32, device=dev)
+        t_route = _time_ms(torch, lambda: heta.route(u, kk, out=(dense, local, None, None)))
+        t_attn = _time_ms(torch, lambda: heta.attention(Q, K, V, w.grid, w.win, dense, out=o,
+                                                         workspace=ws))
+        t_head = _time_ms(torch, lambda: heta.uncertainty(X, wv, 0.0, out=u_next))
+        fl = heta.attention_flops(w.B, w.H, w.d, w.N, kk, w.M)
+        hbytes = 2 * w.B * w.N * w.C + 4 * w.C + 4 * w.B * w.N
+        ms = t_route + t_attn + t_head
+        return {"B": w.B, "H": w.H, "N": w.N, "k": kk, "route_ms": t_route,
+                "attention_ms": t_attn, "head_ms": t_head,
+                "tokens_per_s": w.B * w.N / (ms / 1e3),
+                "attention_tflops": fl / (t_attn * 1e9),
+                "head_gbs": hbytes / (t_head * 1e6)}
+
+    for w in (W.WAN22, W.BATCHED):
+        Q, K, V = (randn_bf16(w.B, w.H, w.N, w.d) for _ in range(3))
+        X = randn_bf16(w.B, w.N, w.C)
+        wv = torch.from_numpy(W.make_head(W.scaled(w, B=1, grid=(1, 1, 8)))[1]).to(dev)
+        u = torch.from_numpy(W.make_u(w)).to(dev)
+        res[w.name] = one_step(w, Q, K, V, X, wv, u)
+        del Q, K, V, X
+    sweep = {}
+    for kind in ("uniform", "clustered"):
+        for rho in W.SWEEP_RHOS:
+            w = W.sweep(rho, kind)
+            kk = heta.dense_count(w.N, rho)
+            u = torch.from_numpy(W.make_u(w)).to(dev)
+            dense, _, _, _ = heta.route(u, kk)
+            ws = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, kk),
+                             dtype=torch.uint8, device=dev)
+            t = _time_ms(torch, lambda: heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense,
+                                                        out=out, workspace=ws))
+            fl = heta.attention_flops(w.B, w.H, w.d, w.N, kk, w.M)
+            sweep["%s-rho%.2f" % (kind, rho)] = {"attention_ms": t,
+                                                 "algorithmic_tflops": fl / (t * 1e9)}
+    res["rho_sweep_wan2.1"] = sweep
+    return res
+
+
 def run_heta(args, info):
     import torch
 
@@ -423,6 +496,11 @@ def run_heta(args, info):
                 "attention_ms": ms_n, "algorithmic_tflops": fl_n / (ms_n * 1e9),
                 "speedup_vs_dense": (dense_cmp["ms"] / ms_n) if dense_cmp else None}
         del ws_n
+
+    # ---- the other configurations, timed the same way on fresh inputs -------
+    others = None
+    if not args.no_other_configs and info.rank == 0 and w.name == W.WAN21.name:
+        others = other_configs(heta, torch, dev, d_Q, d_K, d_V, out)
 
     # ---- the paper's own threshold rule, T = mu + c*sigma (Eq. (11)), c = 0.9 --
     thr = None
@@ -599,6 +677,7 @@ def run_heta(args, info):
                           "peak": peaks["hbm_gbs"], "unit": "GB/s"},
         "dense_compare": dense_cmp,
         "window_sweep": win_sweep,
+        "other_configs": others,
         "threshold_mode": thr,
         "route_throughput": route_tp,
         "route_swap": swap,
