@@ -19,12 +19,17 @@ def check_route(heta, u, k):
     import torch
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     d, l, th, m = heta.route(to_dev(u), k, want_thresh=True, want_mask=True, status=st)
+    # the same call without the optional outputs takes the kernel's other
+    # compaction path (no mask stores)
+    d2, l2, _, _ = heta.route(to_dev(u), k, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     od, ol, om = oracle.route(u, k)
     assert np.array_equal(d.cpu().numpy(), od)
     assert np.array_equal(l.cpu().numpy(), ol)
     assert np.array_equal(m.cpu().numpy(), om)
+    assert np.array_equal(d2.cpu().numpy(), od)
+    assert np.array_equal(l2.cpu().numpy(), ol)
     th = th.cpu().numpy()
     for b in range(u.shape[0]):
         if k == 0:
@@ -63,7 +68,9 @@ def test_route_extreme_k(gpu_lib, k):
 @pytest.mark.parametrize("N,B,kind", [(1, 1, "u"), (33, 2, "u"), (1001, 3, "u"),
                                       (53248, 1, "ties"), (32760, 2, "equal"),
                                       (4097, 2, "signed_zero"), (5000, 1, "denormal"),
-                                      (1024, 4, "inf")])
+                                      (1024, 4, "inf"), (3001, 3, "offset"),
+                                      (2050, 2, "wide"), (53248, 2, "normal"),
+                                      (777, 5, "few_values")])
 def test_route_edge_inputs(gpu_lib, N, B, kind):
     rng = np.random.default_rng(N * 7 + B)
     if kind == "u":
@@ -76,8 +83,20 @@ def test_route_edge_inputs(gpu_lib, N, B, kind):
         u = rng.choice(np.array([-0.0, 0.0, 1.0, -1.0], np.float32), (B, N))
     elif kind == "denormal":
         u = (rng.integers(-20, 20, (B, N)) * np.float32(1e-45)).astype(np.float32)
-    else:
+    elif kind == "inf":
         u = rng.choice(np.array([np.inf, -np.inf, 0.0, 3.0], np.float32), (B, N))
+    elif kind == "offset":
+        # far from 0 relative to the spread: the two-rounding bucket form
+        u = (np.float32(1e6) + rng.random((B, N), dtype=np.float32)).astype(np.float32)
+    elif kind == "wide":
+        # magnitudes from 1e-30 to 1e30 of both signs
+        u = (rng.choice([-1.0, 1.0], (B, N)) * 10.0 ** rng.uniform(-30, 30, (B, N)))
+        u = u.astype(np.float32)
+    elif kind == "normal":
+        u = rng.standard_normal((B, N)).astype(np.float32)
+    else:
+        # a handful of distinct values: buckets with hundreds of equal tokens
+        u = rng.choice(np.array([0.1, 0.25, 0.5, 0.75], np.float32), (B, N))
     for rho in (0.0, 0.2, 0.5, 1.0):
         check_route(gpu_lib, u, gpu_lib.dense_count(N, rho))
 
@@ -90,3 +109,12 @@ def test_route_nan_sets_status(gpu_lib):
     gpu_lib.route(to_dev(u), 100, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == gpu_lib.HETA_ERR_NONFINITE
+
+
+def test_route_many_samples(gpu_lib):
+    """More samples than SMs: each CTA walks several samples (prefetching the
+    next one into L2), some rows 16-byte aligned and some not (N odd)."""
+    rng = np.random.default_rng(99)
+    for N in (1000, 1001):
+        u = rng.standard_normal((300, N)).astype(np.float32)
+        check_route(gpu_lib, u, gpu_lib.dense_count(N, 0.3))
