@@ -88,7 +88,8 @@ HETA_API heta_status heta_dense_count(int N, double rho, int *k_out);
  *   status_dev device int32, or NULL (see conventions).
  *
  * Requires B >= 1, 1 <= N <= 53248 (one sample's keys live in one SM's
- * shared memory), 0 <= k <= N, B*N < 2^31.  One CTA per sample.
+ * shared memory), 0 <= k <= N, B*N < 2^31.  One CTA per sample; for
+ * B <= 8 a cluster of eight CTAs per sample (the same lists, lower latency).
  */
 HETA_API heta_status heta_route(const float *u, int B, int N, int k,
                        int32_t *dense_idx, int32_t *local_idx,

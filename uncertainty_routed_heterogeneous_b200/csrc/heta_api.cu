@@ -54,6 +54,10 @@ heta_status heta_route(const float *u, int B, int N, int k, int32_t *dense_idx,
         (local_idx && !aligned16(local_idx)) || (thresh_out && !aligned16(thresh_out)) ||
         (mask_out && !aligned16(mask_out)))
         return HETA_ERR_INVALID_ARG;
+    if (heta::route_cluster_fits(B, N))
+        return from_cuda(heta::launch_route_cluster(u, B, N, k, dense_idx, local_idx, thresh_out,
+                                                    mask_out, status_dev,
+                                                    static_cast<cudaStream_t>(stream)));
     return from_cuda(heta::launch_route(u, B, N, k, dense_idx, local_idx, thresh_out,
                                         mask_out, status_dev,
                                         static_cast<cudaStream_t>(stream)));

@@ -22,6 +22,15 @@ cudaError_t launch_route(const float *u, int B, int N, int k, int32_t *dense_idx
                          int32_t *local_idx, float *thresh, uint8_t *mask,
                          int32_t *status, cudaStream_t s);
 
+// Up to this many samples, heta_route splits each sample over a cluster of
+// eight CTAs (route_cluster.cu) instead of one CTA (route.cu): the same
+// lists, with the latency of a single sample cut roughly by the split.
+constexpr int kRouteClusterMaxB = 8;
+bool route_cluster_fits(int B, int N);
+cudaError_t launch_route_cluster(const float *u, int B, int N, int k, int32_t *dense_idx,
+                                 int32_t *local_idx, float *thresh, uint8_t *mask,
+                                 int32_t *status, cudaStream_t s);
+
 cudaError_t launch_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
                               uint64_t seed, int block, int32_t *dense_out, int32_t *local_out,
                               uint8_t *mask, int32_t *status, cudaStream_t st);
