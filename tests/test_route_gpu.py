@@ -118,3 +118,19 @@ def test_route_many_samples(gpu_lib):
     for N in (1000, 1001):
         u = rng.standard_normal((300, N)).astype(np.float32)
         check_route(gpu_lib, u, gpu_lib.dense_count(N, 0.3))
+
+
+@pytest.mark.parametrize("N", [33, 4097, 32760, 53248])
+def test_route_cluster_and_single_cta_agree(gpu_lib, N):
+    """Up to eight samples a call split each sample over a cluster of CTAs;
+    more samples take one CTA each.  The same rows routed in a call of 8
+    samples and in a call of 9 give the same lists, and the oracle's."""
+    rng = np.random.default_rng(N)
+    u = rng.standard_normal((9, N)).astype(np.float32)
+    u[3] = rng.integers(0, 5, N).astype(np.float32)  # heavy ties: the key select
+    k = gpu_lib.dense_count(N, 0.2)
+    d9, l9, _, _ = gpu_lib.route(to_dev(u), k)
+    d8, l8, _, _ = gpu_lib.route(to_dev(u[:8].copy()), k)
+    od, ol, _ = oracle.route(u, k)
+    assert np.array_equal(d9.cpu().numpy(), od) and np.array_equal(l9.cpu().numpy(), ol)
+    assert np.array_equal(d8.cpu().numpy(), od[:8]) and np.array_equal(l8.cpu().numpy(), ol[:8])
