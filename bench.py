@@ -558,7 +558,24 @@ def run_heta(args, info):
             heta.route_swap(dense, w.N, s_sw, 2024, blk, out=(sw_d, sw_l, None))
         e1.record()
         torch.cuda.synchronize()
-        swap = {"r": 0.07, "s": s_sw, "us_per_block": 1e3 * e0.elapsed_time(e1) / reps}
+        us_one = 1e3 * e0.elapsed_time(e1) / reps
+        # all 30 blocks of a step (Wan2.1-1.3B has 30) in one launch
+        nb = 30
+        bd = torch.empty((nb,) + tuple(dense.shape), dtype=torch.int32, device=dev)
+        bl = torch.empty((nb,) + tuple(local.shape), dtype=torch.int32, device=dev)
+        for _ in range(3):
+            heta.route_swap_blocks(dense, w.N, s_sw, 2024, 0, nb, out=(bd, bl, None))
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(5):
+            heta.route_swap_blocks(dense, w.N, s_sw, 2024, 0, nb, out=(bd, bl, None))
+        e1.record()
+        torch.cuda.synchronize()
+        us_all = 1e3 * e0.elapsed_time(e1) / 5
+        swap = {"r": 0.07, "s": s_sw, "us_per_block": us_one,
+                "blocks_in_one_launch": nb, "us_all_blocks": us_all,
+                "us_per_block_batched": us_all / nb}
+        del bd, bl
 
     # ---- routing in throughput mode: 512 samples of this N in one launch -------
     route_tp = None

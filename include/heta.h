@@ -127,6 +127,27 @@ HETA_API heta_status heta_route_swap(const int32_t *dense_idx, int B, int N, int
                                      int32_t *status_dev, void *stream);
 
 /*
+ * heta_route_swap_blocks -- heta_route_swap for nblocks consecutive
+ * transformer blocks block0 .. block0 + nblocks - 1 in one launch (one CTA
+ * per sample and block).  Every block's swap starts from the same routing, so
+ * a denoising step can draw all of its blocks' routings at once instead of one
+ * launch a block.  Block block0 + j of sample b writes row j*B + b of each
+ * output:
+ *
+ *   dense_out  [nblocks,B,k] int32 out; local_out [nblocks,B,N-k] int32 out;
+ *   mask_out   [nblocks,B,N] uint8 out, or NULL.
+ *
+ * Identical, block for block, to heta_route_swap.  Requires nblocks >= 1,
+ * block0 + nblocks - 1 <= INT32_MAX, B*N*nblocks < 2^31 and, when
+ * nblocks > 1, dense_out not overlapping dense_idx; else as heta_route_swap.
+ */
+HETA_API heta_status heta_route_swap_blocks(const int32_t *dense_idx, int B, int N, int k,
+                                            int s, uint64_t seed, int block0, int nblocks,
+                                            int32_t *dense_out, int32_t *local_out,
+                                            uint8_t *mask_out, int32_t *status_dev,
+                                            void *stream);
+
+/*
  * heta_route_threshold -- routing by the paper's own rule (Eq. (11)-(12)):
  * per sample b, T_b = mu_b + c * sigma_b, where mu_b and sigma_b are the mean
  * and the population standard deviation of u[b,:], computed in fp64; token i

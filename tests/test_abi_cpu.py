@@ -36,7 +36,7 @@ def test_header_declares_the_three_path_calls():
     assert {"heta_route", "heta_attention", "heta_uncertainty", "heta_dense_count",
             "heta_status_string", "heta_version", "heta_attention_workspace_size",
             "heta_route_threshold", "heta_attention_counts", "heta_route_swap",
-            "heta_attention_counts_workspace_size"} <= names
+            "heta_route_swap_blocks", "heta_attention_counts_workspace_size"} <= names
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -162,6 +162,31 @@ def test_swap_entry_point_validates_on_the_host(lib):
     assert sw(*odd) == heta.HETA_ERR_INVALID_ARG
     assert heta.swap_count(32760, 6552, 0.07) == 2294
     assert heta.swap_count(100, 5, 0.07) == 5
+
+
+def test_swap_blocks_entry_point_validates_on_the_host(lib):
+    """The many-block swap: block count, block range and the rule that the
+    outputs of more than one block may not overlap the input."""
+    N = None
+    base = 1 << 20
+    fake = ctypes.c_void_p(base)
+    sw = lib.heta_route_swap_blocks
+    sw.argtypes = [ctypes.c_void_p] + [ctypes.c_int] * 4 + [ctypes.c_uint64] + \
+        [ctypes.c_int] * 2 + [ctypes.c_void_p] * 5
+    # B=1, N=100, k=20, s=5; input at base, outputs far away
+    far = ctypes.c_void_p(base + (1 << 24))
+    ok = [fake, 1, 100, 20, 5, 7, 0, 3, far, far, N, N, N]
+    for pos, bad in ((7, 0), (7, -2), (6, -1), (4, 21)):
+        a = list(ok)
+        a[pos] = bad
+        assert sw(*a) == heta.HETA_ERR_INVALID_ARG, (pos, bad)
+    a = list(ok)
+    a[6] = 2 ** 31 - 2  # block0 + nblocks - 1 past INT32_MAX
+    assert sw(*a) == heta.HETA_ERR_INVALID_ARG
+    # dense_out overlapping dense_idx with nblocks > 1 (never launched)
+    over = list(ok)
+    over[8] = ctypes.c_void_p(base + 16 * 3)
+    assert sw(*over) == heta.HETA_ERR_INVALID_ARG
 
 
 def test_flop_model_matches_the_papers_reduction():

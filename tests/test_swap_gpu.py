@@ -72,3 +72,30 @@ def test_swap_bad_index_is_reported(gpu_lib):
     heta.route_swap(d, 100, 2, seed=3, block=0, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == heta.HETA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("N,k,s,B", [(32760, 6552, 2294, 2), (1001, 300, 77, 3)])
+def test_swap_blocks_matches_one_block_calls(gpu_lib, N, k, s, B):
+    """All 30 blocks of a step in one launch (heta_route_swap_blocks) give,
+    block for block, the lists of 30 single-block calls; blocks 0 and 29 are
+    also checked against the oracle."""
+    import torch
+    heta = gpu_lib
+    rng = np.random.default_rng(N + B)
+    u = rng.standard_normal((B, N)).astype(np.float32)
+    dense, _, _, _ = heta.route(to_dev(u), k)
+    seed, block0, nb = 0xABCDEF0123456789, 5, 30
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    all_d, all_l, all_m = heta.route_swap_blocks(dense, N, s, seed, block0, nb, want_mask=True,
+                                                 status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for j in range(nb):
+        d1, l1, m1 = heta.route_swap(dense, N, s, seed, block0 + j, want_mask=True)
+        assert torch.equal(all_d[j], d1) and torch.equal(all_l[j], l1)
+        assert torch.equal(all_m[j], m1)
+    dn = dense.cpu().numpy()
+    for j in (0, nb - 1):
+        want_d, want_l = oracle.route_swap(dn, N, s, seed, block0 + j)
+        assert np.array_equal(all_d[j].cpu().numpy(), want_d)
+        assert np.array_equal(all_l[j].cpu().numpy(), want_l)

@@ -70,6 +70,9 @@ def load():
     lib.heta_selftest_wait_timeout.restype = i
     lib.heta_route_swap.argtypes = [vp, i, i, i, i, ctypes.c_uint64, i, vp, vp, vp, vp, vp]
     lib.heta_route_swap.restype = i
+    lib.heta_route_swap_blocks.argtypes = [vp, i, i, i, i, ctypes.c_uint64, i, i, vp, vp, vp,
+                                           vp, vp]
+    lib.heta_route_swap_blocks.restype = i
     lib.heta_route_threshold.argtypes = [vp, i, i, d, vp, vp, vp, vp, vp, vp, vp]
     lib.heta_route_threshold.restype = i
     lib.heta_attention_counts.argtypes = ([vp, vp, vp] + [i] * 9 +
@@ -187,6 +190,35 @@ def route_swap(dense_idx, N: int, s: int, seed: int, block: int, *, out=None, wa
                                 _opt(dense) if k > 0 else None, _opt(local) if k < N else None,
                                 _opt(mask), _opt(status), _stream())
     _check(rc, "heta_route_swap")
+    return dense, local, mask
+
+
+def route_swap_blocks(dense_idx, N: int, s: int, seed: int, block0: int, nblocks: int, *,
+                      out=None, want_mask=False, status=None):
+    """The random swaps of nblocks consecutive transformer blocks in one launch
+    (``heta_route_swap_blocks``).
+
+    dense_idx: [B,k] int32 CUDA.  Returns (dense [nblocks,B,k], local
+    [nblocks,B,N-k], mask [nblocks,B,N] uint8 or None); ``out`` may pass
+    preallocated (dense, local, mask), not overlapping dense_idx.
+    """
+    import torch
+    pd = _dev(dense_idx, torch.int32, "dense_idx", 2)
+    B, k = dense_idx.shape
+    nb = int(nblocks)
+    if out is None:
+        dev = dense_idx.device
+        dense = torch.empty((nb, B, k), dtype=torch.int32, device=dev)
+        local = torch.empty((nb, B, N - k), dtype=torch.int32, device=dev)
+        mask = torch.empty((nb, B, N), dtype=torch.uint8, device=dev) if want_mask else None
+    else:
+        dense, local, mask = out
+    rc = load().heta_route_swap_blocks(pd if k > 0 else None, B, int(N), k, int(s),
+                                       int(seed) & 0xFFFFFFFFFFFFFFFF, int(block0), nb,
+                                       _opt(dense) if k > 0 else None,
+                                       _opt(local) if k < N else None, _opt(mask),
+                                       _opt(status), _stream())
+    _check(rc, "heta_route_swap_blocks")
     return dense, local, mask
 
 

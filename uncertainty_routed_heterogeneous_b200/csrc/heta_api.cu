@@ -63,22 +63,41 @@ heta_status heta_route(const float *u, int B, int N, int k, int32_t *dense_idx,
                                         static_cast<cudaStream_t>(stream)));
 }
 
-heta_status heta_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
-                            uint64_t seed, int block, int32_t *dense_out, int32_t *local_out,
-                            uint8_t *mask_out, int32_t *status_dev, void *stream)
+heta_status heta_route_swap_blocks(const int32_t *dense_idx, int B, int N, int k, int s,
+                                   uint64_t seed, int block0, int nblocks, int32_t *dense_out,
+                                   int32_t *local_out, uint8_t *mask_out, int32_t *status_dev,
+                                   void *stream)
 {
     if (B < 1 || N < 1 || k < 0 || k > N) return HETA_ERR_INVALID_ARG;
-    if (s < 0 || s > k || s > N - k || block < 0) return HETA_ERR_INVALID_ARG;
-    if ((int64_t)B * N >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
+    if (s < 0 || s > k || s > N - k || block0 < 0 || nblocks < 1) return HETA_ERR_INVALID_ARG;
+    if ((int64_t)block0 + nblocks - 1 > INT32_MAX) return HETA_ERR_INVALID_ARG;
+    if ((int64_t)B * N * nblocks >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
+    if ((int64_t)B * nblocks > INT32_MAX) return HETA_ERR_INVALID_ARG;
     if (N > heta::kRouteMaxN) return HETA_ERR_UNSUPPORTED;
     if ((k > 0 && (!dense_idx || !dense_out)) || (k < N && !local_out))
         return HETA_ERR_INVALID_ARG;
     if ((dense_idx && !aligned16(dense_idx)) || (dense_out && !aligned16(dense_out)) ||
         (local_out && !aligned16(local_out)) || (mask_out && !aligned16(mask_out)))
         return HETA_ERR_INVALID_ARG;
-    return from_cuda(heta::launch_route_swap(dense_idx, B, N, k, s, seed, block, dense_out,
-                                             local_out, mask_out, status_dev,
+    if (nblocks > 1 && k > 0) {
+        // the input must not be overwritten while another block still reads it
+        const uintptr_t in0 = reinterpret_cast<uintptr_t>(dense_idx);
+        const uintptr_t in1 = in0 + sizeof(int32_t) * (size_t)B * k;
+        const uintptr_t out0 = reinterpret_cast<uintptr_t>(dense_out);
+        const uintptr_t out1 = out0 + sizeof(int32_t) * (size_t)B * k * nblocks;
+        if (in0 < out1 && out0 < in1) return HETA_ERR_INVALID_ARG;
+    }
+    return from_cuda(heta::launch_route_swap(dense_idx, B, N, k, s, seed, block0, nblocks,
+                                             dense_out, local_out, mask_out, status_dev,
                                              static_cast<cudaStream_t>(stream)));
+}
+
+heta_status heta_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
+                            uint64_t seed, int block, int32_t *dense_out, int32_t *local_out,
+                            uint8_t *mask_out, int32_t *status_dev, void *stream)
+{
+    return heta_route_swap_blocks(dense_idx, B, N, k, s, seed, block, 1, dense_out, local_out,
+                                  mask_out, status_dev, stream);
 }
 
 heta_status heta_route_threshold(const float *u, int B, int N, double c, int32_t *counts,

@@ -32,8 +32,9 @@ cudaError_t launch_route_cluster(const float *u, int B, int N, int k, int32_t *d
                                  int32_t *status, cudaStream_t s);
 
 cudaError_t launch_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
-                              uint64_t seed, int block, int32_t *dense_out, int32_t *local_out,
-                              uint8_t *mask, int32_t *status, cudaStream_t st);
+                              uint64_t seed, int block0, int nblocks, int32_t *dense_out,
+                              int32_t *local_out, uint8_t *mask, int32_t *status,
+                              cudaStream_t st);
 
 cudaError_t launch_route_threshold(const float *u, int B, int N, double c, int32_t *counts,
                                    int32_t *dense_idx, int32_t *local_idx, double *thresh,

@@ -10,7 +10,7 @@
 // local and of the local set the s tokens with the smallest (rho_i, i) go
 // dense, so the count stays k.
 //
-// One CTA per sample: the dense set becomes a bitmap in shared memory, the
+// One CTA per (sample, block): the dense set becomes a bitmap in shared memory, the
 // draws are computed once into shared memory, each set's s smallest draws
 // are found by the same three-pass radix select as the top-k routing (on the
 // complemented draws, so "largest" means smallest), and a ballot compaction
@@ -46,10 +46,15 @@ __device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint3
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-route_swap_kernel(const int32_t *dense_idx, int N, int k, int s, uint32_t seed_lo,
-                  uint32_t seed_hi, int block, int32_t *dense_out, int32_t *local_out,
+route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t seed_lo,
+                  uint32_t seed_hi, int block0, int32_t *dense_out, int32_t *local_out,
                   uint8_t *__restrict__ mask, int32_t *status)
 {
+    // blockIdx.x = beta * B + b: sample b at transformer block block0 + beta;
+    // the outputs of block beta start at beta * B rows
+    const int b = blockIdx.x % B;
+    const int beta = blockIdx.x / B;
+    const int block = block0 + beta;
     extern __shared__ uint32_t dyn[];
     uint32_t *key = dyn;       // [N] complemented draws: larger key = smaller draw
     uint32_t *bits = dyn + N;  // [ceil(N/32)] dense set of the input routing
@@ -61,7 +66,6 @@ route_swap_kernel(const int32_t *dense_idx, int N, int k, int s, uint32_t seed_l
     __shared__ int s_bad;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int b = blockIdx.x;
     const int nwords = (N + 31) >> 5;
     if (tid == 0) s_bad = 0;
     for (int w = tid; w < nwords; w += kThreads) bits[w] = 0u;
@@ -197,9 +201,10 @@ route_swap_kernel(const int32_t *dense_idx, int N, int k, int s, uint32_t seed_l
     }
     __syncthreads();
 
-    int32_t *dout = dense_out + (size_t)b * k;
-    int32_t *lout = local_out + (size_t)b * (N - k);
-    uint8_t *mout = mask ? mask + (size_t)b * N : nullptr;
+    const size_t row = (size_t)beta * B + b;
+    int32_t *dout = dense_out + row * k;
+    int32_t *lout = local_out + row * (N - k);
+    uint8_t *mout = mask ? mask + row * N : nullptr;
     uint32_t rd = w_dense_before[warp];
     uint32_t re[2] = {w_before[0][warp], w_before[1][warp]};
     for (int base = seg_lo; base < seg_hi; base += 32) {
@@ -234,16 +239,17 @@ size_t route_swap_smem_bytes(int N)
 }
 
 cudaError_t launch_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
-                              uint64_t seed, int block, int32_t *dense_out, int32_t *local_out,
-                              uint8_t *mask, int32_t *status, cudaStream_t st)
+                              uint64_t seed, int block0, int nblocks, int32_t *dense_out,
+                              int32_t *local_out, uint8_t *mask, int32_t *status,
+                              cudaStream_t st)
 {
     cudaError_t e = cudaFuncSetAttribute(route_swap_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)route_swap_smem_bytes(kRouteMaxN));
     if (e != cudaSuccess) return e;
-    route_swap_kernel<<<B, kThreads, route_swap_smem_bytes(N), st>>>(
-        dense_idx, N, k, s, (uint32_t)seed, (uint32_t)(seed >> 32), block, dense_out, local_out,
-        mask, status);
+    route_swap_kernel<<<(unsigned)((int64_t)B * nblocks), kThreads, route_swap_smem_bytes(N),
+                        st>>>(dense_idx, B, N, k, s, (uint32_t)seed, (uint32_t)(seed >> 32),
+                              block0, dense_out, local_out, mask, status);
     return cudaGetLastError();
 }
 
