@@ -612,7 +612,7 @@ def run_heta(args, info):
     # come back; two device copies of the inputs and outputs alternate.
     e2e = None
     if not args.no_e2e:
-        ke = max(2, min(args.steps, 10))
+        ke = max(2, min(args.steps, 20))
         s_in, s_cmp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
         sets = [dict(Q=d_Q, K=d_K, V=d_V, X=d_X, u=d_u, out=out, un=u_next)]
         sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
