@@ -83,6 +83,19 @@ route_kernel(const float *__restrict__ u, int B, int N, int k,
         auto owns = [&](int q) {
             return q >= q_lo && q < q_hi && ((q - q_lo) & 31) == lane;
         };
+        // 16-byte copies of this lane's whole quads [qa, qe) of the sample at
+        // us into shared memory, as one commit group
+        auto issue_quads = [&](const float *us, int o, int qlo, int qe, int qfirst, int ln) {
+            const uint4 *g4 = reinterpret_cast<const uint4 *>(us - o);
+            for (int q = qlo + ln; q < qe; q += 32) {
+                if (q < qfirst) continue;
+                const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot4 + q);
+                const size_t src = __cvta_generic_to_global(g4 + q);
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src)
+                             : "memory");
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        };
 
         if (tid == 0) {
             s_nan = 0;
@@ -98,17 +111,12 @@ route_kernel(const float *__restrict__ u, int B, int N, int k,
         float mn = kInf, mx = -kInf;
         {
             // every whole quad of the sample in flight at once: 16-byte
-            // asynchronous copies straight into shared memory
-            const uint4 *g4 = reinterpret_cast<const uint4 *>(ub - off);
+            // asynchronous copies straight into shared memory (when N is a
+            // multiple of 4 each warp issued them at the end of the previous
+            // sample, as soon as its own quads were free; see below)
             const int qe = min(q_hi, qb);
-            for (int q = q_lo + lane; q < qe; q += 32) {
-                if (q < qa) continue;
-                const uint32_t dst = (uint32_t)__cvta_generic_to_shared(slot4 + q);
-                const size_t src = __cvta_generic_to_global(g4 + q);
-                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src)
-                             : "memory");
-            }
-            asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+            if (!((N & 3) == 0 && b != (int)blockIdx.x)) issue_quads(ub, off, q_lo, qe, qa, lane);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
             for (int q = q_lo + lane; q < qe; q += 32) {
                 if (q < qa) continue;
                 const uint4 v = slot4[q];
@@ -419,6 +427,14 @@ route_kernel(const float *__restrict__ u, int B, int N, int k,
                     compact<false, false, true>(slot, off, t_lo, t_hi, kst, take, rd, re,
                                                 dout, lout, mout, ku, nl, lane);
             }
+        }
+        // A warp's quads are free once it has compacted them (no other warp
+        // reads them): when every sample has the same quads (N a multiple of
+        // 4, so the same 16-byte phase), the next sample's copies go out now
+        // and overlap the other warps' tails and the next sample's setup.
+        if ((N & 3) == 0 && b + (int)gridDim.x < B) {
+            const float *un = ub + (size_t)gridDim.x * N;
+            issue_quads(un, off, q_lo, min(q_hi, qb), qa, lane);
         }
         __syncthreads();  // shared memory is reused by the next sample
     }
