@@ -577,33 +577,39 @@ def run_heta(args, info):
                 "us_per_block_batched": us_all / nb}
         del bd, bl
 
-    # ---- routing in throughput mode: 512 samples of this N in one launch -------
+    # ---- routing in throughput mode: many samples of this N in one launch ------
+    # 512 samples, and a whole number of samples per SM (4 x the SM count), so
+    # that no SM runs a last sample alone
     route_tp = None
     if not args.no_route_throughput:
-        Bt = 512
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        hbm = load_peaks()["hbm_gbs"]
         g = torch.Generator(device=dev)
         g.manual_seed(7)
-        u_tp = (d_u[:1].repeat(Bt, 1) +
-                1e-3 * torch.randn((Bt, w.N), generator=g, device=dev)).contiguous()
-        dn_tp = torch.empty((Bt, kk), dtype=torch.int32, device=dev)
-        lc_tp = torch.empty((Bt, w.N - kk), dtype=torch.int32, device=dev)
-        for _ in range(3):
-            heta.route(u_tp, kk, out=(dn_tp, lc_tp, None, None))
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 20
-        e0.record()
-        for _ in range(reps):
-            heta.route(u_tp, kk, out=(dn_tp, lc_tp, None, None))
-        e1.record()
-        torch.cuda.synchronize()
-        us = 1e3 * e0.elapsed_time(e1) / reps
-        nbytes = Bt * w.N * 4 * 2  # read u once, write both index lists
-        hbm = load_peaks()["hbm_gbs"]
-        route_tp = {"B": Bt, "N": w.N, "k": kk, "us": us, "bytes": nbytes,
-                    "GB/s": nbytes / (us * 1e3), "frac_of_hbm": nbytes / (us * 1e3) / hbm,
-                    "peak_source": "measured copy bandwidth"}
-        del u_tp, dn_tp, lc_tp
+        runs = {}
+        for Bt in (512, 4 * sms):
+            u_tp = (d_u[:1].repeat(Bt, 1) +
+                    1e-3 * torch.randn((Bt, w.N), generator=g, device=dev)).contiguous()
+            dn_tp = torch.empty((Bt, kk), dtype=torch.int32, device=dev)
+            lc_tp = torch.empty((Bt, w.N - kk), dtype=torch.int32, device=dev)
+            for _ in range(3):
+                heta.route(u_tp, kk, out=(dn_tp, lc_tp, None, None))
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 20
+            e0.record()
+            for _ in range(reps):
+                heta.route(u_tp, kk, out=(dn_tp, lc_tp, None, None))
+            e1.record()
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / reps
+            nbytes = Bt * w.N * 4 * 2  # read u once, write both index lists
+            runs[Bt] = {"B": Bt, "N": w.N, "k": kk, "us": us, "bytes": nbytes,
+                        "GB/s": nbytes / (us * 1e3), "frac_of_hbm": nbytes / (us * 1e3) / hbm}
+            del u_tp, dn_tp, lc_tp
+        route_tp = dict(runs[512])
+        route_tp["full_waves"] = runs[4 * sms]
+        route_tp["peak_source"] = "measured copy bandwidth"
 
     # ---- end to end through the public API with host buffers ----------------
     # Every step copies its inputs from pinned host memory and reads its
