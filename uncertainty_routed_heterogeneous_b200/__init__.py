@@ -17,9 +17,10 @@ import ctypes
 import math
 import os
 
-__all__ = ["load", "HetaError", "dense_count", "route", "attention", "uncertainty",
-           "attention_workspace_size",
-           "status_string", "attention_flops", "LIB_PATH"]
+__all__ = ["load", "HetaError", "dense_count", "route", "route_threshold", "swap_count",
+           "route_swap", "route_swap_blocks", "attention", "attention_counts",
+           "attention_workspace_size", "attention_counts_workspace_size", "uncertainty",
+           "selftest_wait_timeout", "status_string", "attention_flops", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libheta.so")
 
