@@ -167,11 +167,14 @@ HETA_API heta_status heta_route_swap_blocks(const int32_t *dense_idx, int B, int
  *   mask_out   [B,N] uint8 out, or NULL: m_i, 1 = local, 0 = dense.
  *   status_dev device int32, or NULL.
  *
- * The sums run in a fixed order, so repeated calls give identical results;
- * a u within a few fp64 ulps of T may fall on either side compared with
- * another summation order.  Same size limits as heta_route; pointers
- * 16-byte aligned; one CTA per sample.  heta_attention_counts consumes the
- * outputs without a round trip to the host.
+ * The sums run in one fixed order (eight slices of ceil(N/8) tokens, each
+ * summed by a fixed tree, then added in slice order), so repeated calls --
+ * and calls with any batch size -- give identical results; a u within a few
+ * fp64 ulps of T may fall on either side compared with another summation
+ * order.  Same size limits as heta_route; pointers 16-byte aligned.  For
+ * B <= 8 each sample is split over a cluster of eight CTAs, else one CTA per
+ * sample.  heta_attention_counts consumes the outputs without a round trip
+ * to the host.
  */
 HETA_API heta_status heta_route_threshold(const float *u, int B, int N, double c,
                                           int32_t *counts, int32_t *dense_idx,

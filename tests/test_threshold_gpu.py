@@ -153,3 +153,25 @@ def test_attention_counts_full_size_sampled(gpu_lib):
     """The Wan2.1 shape at the paper's c = 0.9 (about 18% dense)."""
     cnt, _ = run_counts(gpu_lib, W.WAN21, 0.9, n_sample=1200)
     assert 0.1 < cnt[0] / W.WAN21.N < 0.3
+
+
+@pytest.mark.parametrize("N", [7, 1001, 32760, 53248])
+def test_threshold_cluster_and_single_cta_agree(gpu_lib, N):
+    """Up to eight samples a call split each sample over a cluster of CTAs,
+    more take one CTA each; both sum the same eight slices in the same order,
+    so the same rows give bit-identical T, counts and lists in a call of 8
+    samples and in a call of 12 (and the oracle's, outside the rounding band)."""
+    import torch
+    heta = gpu_lib
+    u = np.random.default_rng(N).standard_normal((12, N)).astype(np.float32)
+    c12, d12, l12, t12, _ = heta.route_threshold(to_dev(u), 0.9, want_thresh=True)
+    c8, d8, l8, t8, _ = heta.route_threshold(to_dev(u[:8].copy()), 0.9, want_thresh=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(t8.cpu().numpy(), t12.cpu().numpy()[:8])
+    assert np.array_equal(c8.cpu().numpy(), c12.cpu().numpy()[:8])
+    c = c8.cpu().numpy()
+    for b in range(8):
+        assert np.array_equal(d8[b, :c[b]].cpu().numpy(), d12[b, :c[b]].cpu().numpy())
+        assert np.array_equal(l8[b, :N - c[b]].cpu().numpy(), l12[b, :N - c[b]].cpu().numpy())
+    check_threshold(heta, u, 0.9)
+    check_threshold(heta, u[:8].copy(), 0.9)
