@@ -26,7 +26,13 @@ def check_head(heta, X_bits, w, bias):
 
 
 @pytest.mark.parametrize("B,N,C", [(1, 1, 8), (3, 1000, 96), (2, 777, 1536), (1, 64, 16384),
-                                   (2, 300, 3072)])
+                                   (2, 300, 3072),
+                                   # C = 256 U: each lane's weights in registers
+                                   (1, 1, 256), (3, 5, 512), (2, 1001, 768), (1, 4000, 1024),
+                                   (2, 333, 1280), (1, 2500, 1536), (1, 97, 1792),
+                                   (2, 150, 2048), (1, 1201, 2304), (1, 60, 2560),
+                                   (3, 211, 2816), (1, 3000, 3072), (1, 40, 3328),
+                                   (2, 1234, 1544)])
 def test_head_shapes(gpu_lib, B, N, C):
     rng = np.random.default_rng(B * N + C)
     X = W.bf16_bits(rng.standard_normal((B, N, C), dtype=np.float32))
