@@ -314,6 +314,11 @@ HETA_API heta_status heta_attention_noalloc(const uint16_t *Q, const uint16_t *K
  *   u_out  [B,N] fp32 out: the u that routes the next denoising step.
  *
  * Requires B, N >= 1, C a multiple of 8 with 8 <= C <= 16384.
+ *
+ * Widths that are a multiple of 256 up to 3072 (the DiT hidden sizes) run a
+ * kernel that holds each lane's slice of w in registers; other widths stage
+ * w in shared memory.  Both sum the C products in fp32, in an order fixed
+ * by C, so a call is deterministic; the two orders differ only in rounding.
  */
 HETA_API heta_status heta_uncertainty(const uint16_t *X, const float *w, float bias,
                              int B, int N, int C, float *u_out,
