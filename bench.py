@@ -70,6 +70,12 @@ def parse_args():
                    help="mark route / attention / head of every step with NVTX ranges")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="minimum host time the cpu_baseline oracle sample runs for")
+    p.add_argument("--shard", choices=["samples", "heads"], default="samples",
+                   help="samples: each rank runs its own sample (weak scaling, the default); "
+                        "heads: the ranks split one sample's heads and the head's token rows "
+                        "and all-gather the next step's u (strong scaling)")
+    p.add_argument("--gather-out", action="store_true",
+                   help="with --shard heads: also all-gather the output along heads")
     return p.parse_args()
 
 
@@ -112,7 +118,7 @@ class ClockSampler:
         "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
         "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, torch_device_index, period_s=0.01):
+    def __init__(self, torch_device_index, period_s=0.002):
         self.samples = []
         self.period = period_s
         self._stop = threading.Event()
@@ -287,6 +293,66 @@ def config_of(w, n_gpus):
 
 
 # ----------------------------------------------------------------------------
+# parity of the timed output against the fp64 oracle (after the timed region)
+# ----------------------------------------------------------------------------
+
+TOL_MAX_ABS, TOL_MEAN_ABS = 2e-2, 2e-3
+
+
+def parity_rows(w, dense_np, n_per_head, seed):
+    """Flat output row ids (b*H + h)*N + i to check: n_per_head seeded random
+    rows of every (b, h), every border class of the window clamp (the corners,
+    edges and centre of the grid on each axis) in the first and last head, and
+    the first and last three dense rows there."""
+    T, Hg, Wg = w.grid
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for bh in range(w.B * w.H):
+        n = min(n_per_head, w.N)
+        rows.update(int(bh * w.N + i) for i in rng.choice(w.N, size=n, replace=False))
+    edge = []
+    for t in sorted({0, 1, T // 2, T - 2, T - 1}):
+        for h in sorted({0, w.win[1] // 2, Hg // 2, Hg - 1 - w.win[1] // 2, Hg - 1}):
+            for x in sorted({0, w.win[2] // 2, Wg // 2, Wg - 1 - w.win[2] // 2, Wg - 1}):
+                if 0 <= t < T and 0 <= h < Hg and 0 <= x < Wg:
+                    edge.append((t * Hg + h) * Wg + x)
+    for b in range(w.B):
+        for h in sorted({0, w.H - 1}):
+            base = (b * w.H + h) * w.N
+            rows.update(base + i for i in edge)
+            d = dense_np[b]
+            rows.update(base + int(i) for i in d[:3])
+            rows.update(base + int(i) for i in d[-3:])
+    return np.array(sorted(rows), np.int64)
+
+
+def bf16_host_f32(t):
+    """A bf16 tensor (any device) as float32 numpy (exact)."""
+    import torch
+    return W.bf16_to_f32(t.detach().contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def parity_of(w, kk, u_np, q32, k32, v32, dense_t, local_t, out_t, n_per_head, seed):
+    """The routing lists bit for bit, and sampled output rows within the
+    tolerance, against the oracle on the same inputs."""
+    import oracle
+    od, ol, _ = oracle.route(u_np, kk)
+    routing_exact = bool(np.array_equal(dense_t.cpu().numpy(), od) and
+                         (local_t is None or np.array_equal(local_t.cpu().numpy(), ol)))
+    rows = parity_rows(w, od, n_per_head, seed)
+    got = bf16_host_f32(out_t).reshape(-1, w.d)[rows]
+    want = oracle.attention_rows(q32, k32, v32, w.grid, w.win, od, rows)
+    err = np.abs(got.astype(np.float64) - want)
+    mx = float(err.max()) if err.size else 0.0
+    mean = float(err.mean()) if err.size else 0.0
+    return {"max_abs": mx, "mean_abs": mean, "rows": int(rows.size),
+            "rows_per_head": n_per_head, "routing_exact": routing_exact,
+            "within_tolerance": bool(np.all(np.isfinite(got)) and mx <= TOL_MAX_ABS and
+                                     mean <= TOL_MEAN_ABS),
+            "tolerance": {"max_abs": TOL_MAX_ABS, "mean_abs": TOL_MEAN_ABS}}
+
+
+# ----------------------------------------------------------------------------
 # GPU arm
 # ----------------------------------------------------------------------------
 
@@ -315,7 +381,7 @@ def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
     def randn_bf16(*shape):
         return torch.randn(shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
 
-    def one_step(w, Q, K, V, X, wv, u):
+    def one_step(w, Q, K, V, X, wv, u, n_check):
         kk = heta.dense_count(w.N, w.rho)
         dense = torch.empty((w.B, kk), dtype=torch.int32, device=dev)
         local = torch.empty((w.B, w.N - kk), dtype=torch.int32, device=dev)
@@ -330,33 +396,40 @@ def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
         fl = heta.attention_flops(w.B, w.H, w.d, w.N, kk, w.M)
         hbytes = 2 * w.B * w.N * w.C + 4 * w.C + 4 * w.B * w.N
         ms = t_route + t_attn + t_head
+        torch.cuda.synchronize()
+        par = parity_of(w, kk, u.cpu().numpy(), bf16_host_f32(Q), bf16_host_f32(K),
+                        bf16_host_f32(V), dense, local, o, n_check, 5)
         return {"B": w.B, "H": w.H, "N": w.N, "k": kk, "route_ms": t_route,
                 "attention_ms": t_attn, "head_ms": t_head,
                 "tokens_per_s": w.B * w.N / (ms / 1e3),
                 "attention_tflops": fl / (t_attn * 1e9),
-                "head_gbs": hbytes / (t_head * 1e6)}
+                "head_gbs": hbytes / (t_head * 1e6), "parity": par}
 
     for w in (W.WAN22, W.BATCHED):
         Q, K, V = (randn_bf16(w.B, w.H, w.N, w.d) for _ in range(3))
         X = randn_bf16(w.B, w.N, w.C)
         wv = torch.from_numpy(W.make_head(W.scaled(w, B=1, grid=(1, 1, 8)))[1]).to(dev)
         u = torch.from_numpy(W.make_u(w)).to(dev)
-        res[w.name] = one_step(w, Q, K, V, X, wv, u)
+        res[w.name] = one_step(w, Q, K, V, X, wv, u, 256)
         del Q, K, V, X
     sweep = {}
+    q32, k32, v32 = bf16_host_f32(d_Q), bf16_host_f32(d_K), bf16_host_f32(d_V)
     for kind in ("uniform", "clustered"):
         for rho in W.SWEEP_RHOS:
             w = W.sweep(rho, kind)
             kk = heta.dense_count(w.N, rho)
-            u = torch.from_numpy(W.make_u(w)).to(dev)
-            dense, _, _, _ = heta.route(u, kk)
+            u_np = W.make_u(w)
+            u = torch.from_numpy(u_np).to(dev)
+            dense, local, _, _ = heta.route(u, kk)
             ws = torch.empty(heta.attention_workspace_size(w.B, w.H, w.d, w.grid, w.win, kk),
                              dtype=torch.uint8, device=dev)
             t = _time_ms(torch, lambda: heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense,
                                                         out=out, workspace=ws))
             fl = heta.attention_flops(w.B, w.H, w.d, w.N, kk, w.M)
-            sweep["%s-rho%.2f" % (kind, rho)] = {"attention_ms": t,
-                                                 "algorithmic_tflops": fl / (t * 1e9)}
+            torch.cuda.synchronize()
+            sweep["%s-rho%.2f" % (kind, rho)] = {
+                "attention_ms": t, "algorithmic_tflops": fl / (t * 1e9),
+                "parity": parity_of(w, kk, u_np, q32, k32, v32, dense, local, out, 256, 6)}
     res["rho_sweep_wan2.1"] = sweep
     return res
 
@@ -452,6 +525,9 @@ def run_heta(args, info):
     head_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     tokens_per_step = w.B * w.N * info.world
     value = tokens_per_step * args.steps / (ms_total / 1e3)
+    # the last timed step's routing and output, checked against the oracle
+    # once all timing is done
+    timed = (dense.cpu(), local.cpu(), out.cpu())
 
     # ---- our own full dense attention (rho = 1) at the same shape -----------
     dense_cmp = None
@@ -673,6 +749,13 @@ def run_heta(args, info):
     cpu = None
     if info.rank == 0 and info.world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args, base)
+    parity = None
+    if info.rank == 0:
+        parity = parity_of(w, kk, u, bf16_host_f32(h_Q), bf16_host_f32(h_K), bf16_host_f32(h_V),
+                           *timed, 4096, 1)
+        parity["checked"] = ("the last timed step: dense/local lists bit for bit; %d output "
+                             "rows (4096 random per head, every border class and the first "
+                             "and last dense rows) against the fp64 oracle" % parity["rows"])
 
     sampler.close()
     if info.rank != 0:
@@ -708,10 +791,99 @@ def run_heta(args, info):
         "threshold_mode": thr,
         "route_throughput": route_tp,
         "route_swap": swap,
+        "parity": parity,
         "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "cpu_baseline": cpu, "clocks": sampler.summary(),
     }
     line["head_roofline"]["frac"] = line["head_roofline"]["achieved"] / peaks["hbm_gbs"]
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_heta_heads(args, info):
+    """One sample split over the ranks by heads (strong scaling): every rank
+    routes the sample's full u itself, runs attention on its head block and
+    the uncertainty head on its block of token rows; the next step's u, which
+    every rank needs, is all-gathered (NCCL); optionally the output too."""
+    import torch
+
+    import uncertainty_routed_heterogeneous_b200 as heta
+
+    torch.cuda.set_device(info.local_rank)
+    dev = torch.device("cuda", info.local_rank)
+    D.init("nccl", info, timeout_s=300)
+    heta.load()
+    w = chosen_workload(args)
+    if w.B != 1:
+        raise SystemExit("--shard heads takes one sample (B = 1)")
+    if (w.B * w.N) % info.world:
+        raise SystemExit("--shard heads needs the token count divisible by the rank count")
+    h0, h1 = D.head_range(w.H, info.world, info.rank)
+    r0, r1 = D.row_range(w.B * w.N, info.world, info.rank)
+
+    def dev_bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(
+            torch.bfloat16).to(dev)
+
+    q, k, v = W.make_qkv(w)
+    d_Q, d_K, d_V = (dev_bf16(a[:, h0:h1]) for a in (q, k, v))
+    del q, k, v
+    X, wv = W.make_head(w)
+    d_X = dev_bf16(X.reshape(1, w.B * w.N, w.C)[:, r0:r1])
+    del X
+    d_w = torch.from_numpy(wv).to(dev)
+    d_u = torch.from_numpy(W.make_u(w)).to(dev)
+    kk = heta.dense_count(w.N, w.rho)
+    Hl = h1 - h0
+    dense = torch.empty((w.B, kk), dtype=torch.int32, device=dev)
+    local = torch.empty((w.B, w.N - kk), dtype=torch.int32, device=dev)
+    out = torch.empty_like(d_Q)
+    ws = torch.empty(max(256, heta.attention_workspace_size(w.B, Hl, w.d, w.grid, w.win, kk)),
+                     dtype=torch.uint8, device=dev)
+    u_rows = torch.empty((1, r1 - r0), dtype=torch.float32, device=dev)
+    gather_out = args.gather_out and w.H % info.world == 0
+
+    def step():
+        heta.route(d_u, kk, out=(dense, local, None, None))
+        if Hl > 0:
+            heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense, out=out, workspace=ws)
+        heta.uncertainty(d_X, d_w, 0.0, out=u_rows)
+        u_next = D.all_gather_equal(u_rows, info)
+        if gather_out:
+            D.all_gather_equal(out, info)
+        return u_next
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(info.local_rank)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier(info, dev)
+    torch.cuda.synchronize()
+    sampler.start()
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    sampler.stop()
+    D.barrier(info, dev)
+    ms_total = D.max_over_ranks(t0.elapsed_time(t1), info, dev)
+    sampler.close()
+    if info.rank != 0:
+        return 0
+    value = w.B * w.N * args.steps / (ms_total / 1e3)
+    cfg = config_of(w, info.world)
+    cfg["parallelism"] = ("heads%d: one sample's %d heads split over %d GPUs, u of the next "
+                          "step all-gathered%s" % (info.world, w.H, info.world,
+                                                    ", output all-gathered" if gather_out
+                                                    else ""))
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": info.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded; Wan2.1-1.3B latent shape)",
+            "config": cfg, "gpu_launches": (3 if Hl > 0 else 2) * args.steps,
+            "clocks": sampler.summary()}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -721,7 +893,10 @@ def main():
     info = D.rank_info()
     if args.impl == "reference":
         return run_reference(args, info)
-    rc = run_heta(args, info)
+    if args.shard == "heads":
+        rc = run_heta_heads(args, info)
+    else:
+        rc = run_heta(args, info)
     if info.world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -87,9 +87,11 @@ HETA_API heta_status heta_dense_count(int N, double rho, int *k_out);
  *   mask_out   [B,N] uint8 out, or NULL: the paper's m_i, 1 = local, 0 = dense.
  *   status_dev device int32, or NULL (see conventions).
  *
- * Requires B >= 1, 1 <= N <= 53248 (one sample's keys live in one SM's
- * shared memory), 0 <= k <= N, B*N < 2^31.  One CTA per sample; for
- * B <= 8 a cluster of eight CTAs per sample (the same lists, lower latency).
+ * Requires B >= 1, 1 <= N <= 393216, 0 <= k <= N, B*N < 2^31.  A sample
+ * of up to 53248 tokens fits one SM's shared memory: one CTA per sample,
+ * or, for B <= 8, a cluster of eight CTAs per sample (the same lists, lower
+ * latency).  Larger samples (a 720p Wan latent has 75600 tokens) always take
+ * the cluster of eight CTAs, each holding an eighth of the sample.
  */
 HETA_API heta_status heta_route(const float *u, int B, int N, int k,
                        int32_t *dense_idx, int32_t *local_idx,
@@ -118,8 +120,9 @@ HETA_API heta_status heta_route(const float *u, int B, int N, int k,
  *   local_out  [B,N-k] int32 out: the complements, increasing.
  *   mask_out   [B,N] uint8 out, or NULL: m_i of the new sets, 1 = local.
  *
- * Requires 0 <= s <= min(k, N-k), block >= 0 and the heta_route size limits;
- * pointers 16-byte aligned.  One CTA per sample.
+ * Requires 0 <= s <= min(k, N-k), block >= 0, N <= 53248 (one sample in
+ * one SM's shared memory) and B*N < 2^31; pointers 16-byte aligned.  One CTA
+ * per sample.
  */
 HETA_API heta_status heta_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
                                      uint64_t seed, int block, int32_t *dense_out,
@@ -172,8 +175,8 @@ HETA_API heta_status heta_route_swap_blocks(const int32_t *dense_idx, int B, int
  * and calls with any batch size -- give identical results; a u within a few
  * fp64 ulps of T may fall on either side compared with another summation
  * order.  Same size limits as heta_route; pointers 16-byte aligned.  For
- * B <= 8 each sample is split over a cluster of eight CTAs, else one CTA per
- * sample.  heta_attention_counts consumes the outputs without a round trip
+ * B <= 8, or N > 53248, each sample is split over a cluster of eight CTAs,
+ * else one CTA per sample.  heta_attention_counts consumes the outputs without a round trip
  * to the host.
  */
 HETA_API heta_status heta_route_threshold(const float *u, int B, int N, double c,
@@ -184,7 +187,10 @@ HETA_API heta_status heta_route_threshold(const float *u, int B, int N, double c
 
 /*
  * heta_attention_workspace_size -- device scratch one heta_attention call
- * needs for these sizes (host-only; touches no device).
+ * needs for these sizes (host-only; launches nothing).  The dense work is
+ * cut into waves of the current device's multiprocessor count (148 on a
+ * B200, and 148 when no device is visible), so ask with the device current
+ * that the call will run on.
  *
  * The scratch holds the work-item counter of the persistent kernel and, when
  * the pairs of dense query tiles of a last, at most half-full wave of work
@@ -213,8 +219,14 @@ HETA_API heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, 
  *
  *   Q, K, V    [B,H,N,d] bf16, contiguous, read only.
  *   dense_idx  [B,k] int32: D_b, strictly increasing, 0 <= idx < N (the
- *              heta_route output).  Not checked on the device: indices out
- *              of range or out of order give unspecified rows.
+ *              heta_route output).  Every entry is checked on the device:
+ *              an entry outside [0, N), or not greater than the entry before
+ *              it, raises status_dev to HETA_ERR_INVALID_ARG, and the row it
+ *              names is neither read nor written through it.  The rows of the
+ *              sample are then unspecified (a token near a bad entry may get
+ *              its dense result, its local result or no write), but every
+ *              read stays inside Q, K, V and dense_idx and every write inside
+ *              out.
  *   out        [B,H,N,d] bf16 out; every row is written exactly once.
  *   scale      softmax scale, normally 1/sqrt(d).
  *   workspace  device scratch of at least heta_attention_workspace_size()
@@ -256,7 +268,9 @@ HETA_API heta_status heta_attention(const uint16_t *Q, const uint16_t *K,
  */
 /*
  * heta_attention_counts_workspace_size -- device scratch one
- * heta_attention_counts call needs (host-only).  It covers whatever counts
+ * heta_attention_counts call needs (host-only; like
+ * heta_attention_workspace_size it depends on the current device's
+ * multiprocessor count).  It covers whatever counts
  * the device finds (at most ~40 MB at d = 128; 256 bytes when the key range
  * is too short to split).  Same argument rules as heta_attention_counts.
  */
@@ -287,9 +301,18 @@ HETA_API heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K,
  * the scratch heta_attention would use (heta_attention_workspace_size)
  * exceeds 16 MiB, no dense pair is cut into key ranges: the kernel then needs
  * only its work counter, and the result is the same up to rounding order
- * (a partly filled last wave of dense work takes longer).  The first call on each device looks up the array's device
- * address (a host-side runtime query, done once per device with that device
- * current), so make the first call on a device before any stream capture.
+ * (a partly filled last wave of dense work takes longer).
+ *
+ * The first call on a device loads the part of the library that holds the
+ * array, and the driver commits the 16 MiB at that moment (with CUDA's
+ * default lazy module loading; eagerly loaded, at library load).  That first
+ * call can therefore block in the driver's allocator, or fail with
+ * HETA_ERR_CUDA on a full device, so make it a warm-up call outside any
+ * region that must not allocate, and before any stream capture.  It also
+ * looks up the array's device address (a host-side runtime query, with that
+ * device current); the address is remembered per device and context and
+ * looked up again when another context is current (a new primary context
+ * after cudaDeviceReset loads the module, and commits the array, anew).
  * All calls share the array and it keeps the last call's contents; each call
  * clears what must start at zero.  Calls whose kernels may overlap on the
  * GPU (unordered streams) race on the array: order them.

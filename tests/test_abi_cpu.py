@@ -69,7 +69,7 @@ def test_host_validation_returns_before_any_launch(lib):
     assert lib.heta_route(N, 1, 10, 11, N, N, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
     assert lib.heta_route(N, 1, 10, 2, N, N, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
     fake = ctypes.c_void_p(1 << 20)
-    assert lib.heta_route(fake, 1, 60000, 2, fake, fake, N, N, N, N) == \
+    assert lib.heta_route(fake, 1, 8 * 49152 + 1, 2, fake, fake, N, N, N, N) == \
         heta.HETA_ERR_UNSUPPORTED
     # misaligned pointer
     odd = ctypes.c_void_p((1 << 20) + 4)
@@ -111,7 +111,7 @@ def test_threshold_entry_points_validate_on_the_host(lib):
     rt.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, d] + [ctypes.c_void_p] * 7
     assert rt(fake, 0, 10, d(0.9), fake, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
     assert rt(fake, 1, 0, d(0.9), fake, fake, fake, N, N, N, N) == heta.HETA_ERR_INVALID_ARG
-    assert rt(fake, 1, 60000, d(0.9), fake, fake, fake, N, N, N, N) == \
+    assert rt(fake, 1, 8 * 49152 + 1, d(0.9), fake, fake, fake, N, N, N, N) == \
         heta.HETA_ERR_UNSUPPORTED
     assert rt(fake, 1, 10, d(float("nan")), fake, fake, fake, N, N, N, N) == \
         heta.HETA_ERR_INVALID_ARG

@@ -69,7 +69,7 @@ def test_multi_tile_all_rows(gpu_lib, w, rho):
 
 
 @pytest.mark.parametrize("name", ["wan2.1-1.3b-21x30x52", "wan2.2-5b-31x22x40",
-                                  "wan2.1-1.3b-batched-b2"])
+                                  "wan2.1-1.3b-batched-b2", "wan2.1-1.3b-720p-21x45x80"])
 def test_full_size_sampled_rows(gpu_lib, name):
     """4096 random rows per head on average, plus every border-clamped window
     class and the first and last dense rows of the first and last head."""
@@ -145,3 +145,92 @@ def test_degenerate_cases(gpu_lib, case):
         got = from_dev_bf16(out)[0][:, loc]
         want = W.bf16_to_f32(v)[0][:, loc]
         assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# A routing list that breaks the contract (Eq. (12)-(13): the dense set is a
+# subset of the sample's N tokens, listed in increasing order).  Q, K, V and
+# out live inside larger buffers with guard rows before and after, so an
+# access the kernel should not make lands in memory the test owns and checks.
+# ---------------------------------------------------------------------------
+
+_GUARD = 64  # rows of d values before and after each tensor
+_SENTINEL = 0x7FC1  # a bf16 NaN pattern the kernel never writes
+
+
+def _guarded(bits, B, H, N, d):
+    """bf16 bits [B,H,N,d] placed inside a [B*H*N + 2*_GUARD, d] device buffer."""
+    import torch
+    total = B * H * N + 2 * _GUARD
+    host = np.full((total, d), _SENTINEL, np.uint16)
+    if bits is not None:
+        host[_GUARD:_GUARD + B * H * N] = bits.reshape(-1, d)
+    buf = torch.from_numpy(host.view(np.int16)).view(torch.bfloat16).cuda()
+    view = buf[_GUARD:_GUARD + B * H * N].view(B, H, N, d)
+    return buf, view
+
+
+def _noalloc_call(heta, Q, K, V, grid, win, dense, out, st):
+    import ctypes
+    import math
+    import torch
+    fn = heta.load().heta_attention_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.argtypes = [vp, vp, vp] + [i] * 9 + [ctypes.c_float, vp, i, vp, vp, vp]
+    fn.restype = i
+    B, H, N, d = Q.shape
+    rc = fn(vp(Q.data_ptr()), vp(K.data_ptr()), vp(V.data_ptr()), B, H, d, *grid, *win,
+            ctypes.c_float(1.0 / math.sqrt(d)), vp(dense.data_ptr()), dense.shape[1],
+            vp(out.data_ptr()), vp(st.data_ptr()),
+            vp(torch.cuda.current_stream().cuda_stream))
+    assert rc == heta.HETA_OK, heta.status_string(rc)
+
+
+@pytest.mark.parametrize("entry", ["attention", "attention_counts", "attention_noalloc"])
+def test_bad_dense_idx_is_reported_and_stays_in_bounds(gpu_lib, entry):
+    """Sample 0's list starts with -1 and sample 2's ends with N + 5 (both
+    still increasing); sample 1's holds N in the middle and one swapped pair.
+    The status must read HETA_ERR_INVALID_ARG, no guard row of out may
+    change, samples 0 and 2 must equal the oracle with the bad entries left
+    out (their tokens get the local result), and the key range of the dense
+    rows is split in two (N = 2560), so both halves check their rows."""
+    import torch
+    heta = gpu_lib
+    w = dataclasses.replace(W.scaled(W.WAN21, B=3, H=2, d=128, grid=(4, 16, 40),
+                                     win=(3, 5, 7), u_kind="uniform", u_seeds=(31, 32, 33)),
+                            name="bad-dense-idx")
+    B, H, N, d = w.B, w.H, w.N, w.d
+    q, k, v = W.make_qkv(w)
+    u = W.make_u(w)
+    kk = heta.dense_count(N, 0.2)
+    od, _, _ = oracle.route(u, kk)
+    bad = od.copy()
+    bad[0, 0] = -1
+    bad[2, kk - 1] = N + 5
+    bad[1, 100] = N
+    bad[1, 200], bad[1, 201] = od[1, 201], od[1, 200]
+    qb, Qd = _guarded(q, B, H, N, d)
+    kb, Kd = _guarded(k, B, H, N, d)
+    vb, Vd = _guarded(v, B, H, N, d)
+    ob, out = _guarded(None, B, H, N, d)
+    out.fill_(float("nan"))
+    dense = to_dev(bad)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if entry == "attention":
+        heta.attention(Qd, Kd, Vd, w.grid, w.win, dense, out=out, status=st)
+    elif entry == "attention_counts":
+        counts = torch.full((B,), kk, dtype=torch.int32, device="cuda")
+        heta.attention_counts(Qd, Kd, Vd, w.grid, w.win, dense, counts, out=out, status=st)
+    else:
+        _noalloc_call(heta, Qd, Kd, Vd, w.grid, w.win, dense, out, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == heta.HETA_ERR_INVALID_ARG
+    raw = ob.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.all(raw[:_GUARD] == _SENTINEL), "a row before out was written"
+    assert np.all(raw[_GUARD + B * H * N:] == _SENTINEL), "a row after out was written"
+    got = from_dev_bf16(out)
+    qf, kf, vf = W.bf16_to_f32(q), W.bf16_to_f32(k), W.bf16_to_f32(v)
+    for b, keep in ((0, od[0, 1:]), (2, od[2, :kk - 1])):
+        want = oracle.attention(qf[b:b + 1], kf[b:b + 1], vf[b:b + 1], w.grid, w.win,
+                                keep[None, :])
+        assert_close(got[b:b + 1].reshape(-1, d), want.reshape(-1, d), "sample %d" % b)

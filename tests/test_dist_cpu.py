@@ -86,3 +86,62 @@ def test_a_rank_that_dies_ends_the_others_collective_with_an_error():
     assert what != "no error"
     assert secs < 60
     assert procs[1].exitcode == 3
+
+
+def _worker_heads(rank, world, port, q):
+    """One sample split by heads: each rank computes its head block of the
+    attention and its token rows of the uncertainty head with the oracle, then
+    the blocks are gathered the way the head-sharded bench step gathers them."""
+    import numpy as np
+    import torch
+
+    import oracle
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    info = D.rank_info()
+    D.init("gloo", info, timeout_s=30)
+    w = W.scaled(W.WAN21, H=4, d=64, grid=(3, 8, 10), win=(3, 5, 5), u_kind="uniform",
+                 u_seeds=(41,), C=64)
+    q_, k_, v_ = (W.bf16_to_f32(a) for a in W.make_qkv(w))
+    u = W.make_u(w)
+    X, wv = W.make_head(w)
+    X = W.bf16_to_f32(X)
+    kk = oracle.dense_count(w.N, w.rho)
+    dense, _, _ = oracle.route(u, kk)  # every rank routes the same u itself
+    h0, h1 = D.head_range(w.H, world, rank)
+    out = oracle.attention(q_[:, h0:h1], k_[:, h0:h1], v_[:, h0:h1], w.grid, w.win, dense)
+    r0, r1 = D.row_range(w.B * w.N, world, rank)
+    u_next = oracle.uncertainty(X.reshape(1, -1, w.C)[:, r0:r1], wv)
+    out_all = D.all_gather_equal(torch.from_numpy(np.ascontiguousarray(out)), info)
+    u_all = D.all_gather_equal(torch.from_numpy(np.ascontiguousarray(u_next)), info)
+    q.put((rank, out_all.numpy(), u_all.numpy()))
+    import torch.distributed as dist
+    dist.destroy_process_group()
+
+
+def test_head_sharded_step_gathers_to_the_single_rank_result():
+    import numpy as np
+
+    import oracle
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker_heads, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=180) for _ in procs), key=lambda x: x[0])
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    w = W.scaled(W.WAN21, H=4, d=64, grid=(3, 8, 10), win=(3, 5, 5), u_kind="uniform",
+                 u_seeds=(41,), C=64)
+    q_, k_, v_ = (W.bf16_to_f32(a) for a in W.make_qkv(w))
+    u = W.make_u(w)
+    X, wv = W.make_head(w)
+    kk = oracle.dense_count(w.N, w.rho)
+    dense, _, _ = oracle.route(u, kk)
+    want_out = oracle.attention(q_, k_, v_, w.grid, w.win, dense)
+    want_u = oracle.uncertainty(W.bf16_to_f32(X), wv)
+    for _, out_all, u_all in res:
+        assert np.array_equal(out_all.reshape(want_out.shape), want_out)
+        assert np.array_equal(u_all.reshape(want_u.shape), want_u)

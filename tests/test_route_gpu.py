@@ -39,7 +39,7 @@ def check_route(heta, u, k):
 
 
 @pytest.mark.parametrize("name", ["tiny-4x8x8", "wan2.1-1.3b-21x30x52", "wan2.2-5b-31x22x40",
-                                  "wan2.1-1.3b-batched-b2"])
+                                  "wan2.1-1.3b-batched-b2", "wan2.1-1.3b-720p-21x45x80"])
 def test_route_workloads(gpu_lib, name):
     w = W.ALL[name]
     u = W.make_u(w)
@@ -134,3 +134,25 @@ def test_route_cluster_and_single_cta_agree(gpu_lib, N):
     od, ol, _ = oracle.route(u, k)
     assert np.array_equal(d9.cpu().numpy(), od) and np.array_equal(l9.cpu().numpy(), ol)
     assert np.array_equal(d8.cpu().numpy(), od[:8]) and np.array_equal(l8.cpu().numpy(), ol[:8])
+
+
+@pytest.mark.parametrize("N,B", [(53249, 1), (75600, 1), (75600, 9), (75601, 3),
+                                 (8 * 49152, 1)])
+def test_route_above_one_cta(gpu_lib, N, B):
+    """Samples too large for one SM's shared memory (53248 tokens) take the
+    cluster kernel whatever the batch size: the 720p Wan latent (75600), a
+    ragged size, more samples than one cluster a call, and the largest N."""
+    rng = np.random.default_rng(N + B)
+    u = rng.standard_normal((B, N)).astype(np.float32)
+    if B > 1:
+        u[1] = rng.integers(0, 9, N).astype(np.float32)  # heavy ties: the key select
+    for rho in (0.0, 0.2, 1.0):
+        check_route(gpu_lib, u, gpu_lib.dense_count(N, rho))
+
+
+def test_route_above_the_limit_is_unsupported(gpu_lib):
+    import torch
+    u = torch.zeros((1, 8 * 49152 + 1), dtype=torch.float32, device="cuda")
+    with pytest.raises(gpu_lib.HetaError) as e:
+        gpu_lib.route(u, 10)
+    assert e.value.code == gpu_lib.HETA_ERR_UNSUPPORTED

@@ -175,3 +175,13 @@ def test_threshold_cluster_and_single_cta_agree(gpu_lib, N):
         assert np.array_equal(l8[b, :N - c[b]].cpu().numpy(), l12[b, :N - c[b]].cpu().numpy())
     check_threshold(heta, u, 0.9)
     check_threshold(heta, u[:8].copy(), 0.9)
+
+
+@pytest.mark.parametrize("N,B", [(75600, 1), (75600, 9), (8 * 49152, 2)])
+def test_threshold_above_one_cta(gpu_lib, N, B):
+    """Samples above one SM's shared memory (53248 tokens; the 720p Wan latent
+    has 75600) take the cluster kernel for any batch size."""
+    rng = np.random.default_rng(N - B)
+    u = rng.standard_normal((B, N)).astype(np.float32)
+    for c in (0.0, 0.9):
+        check_threshold(gpu_lib, u, c)

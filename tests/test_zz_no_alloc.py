@@ -3,10 +3,16 @@
 Some callers cannot allocate device memory (no cudaMalloc allowed where they
 run), so they cannot hand heta_attention a workspace.  heta_attention_noalloc
 takes the same arguments minus the workspace and keeps its scratch in a fixed
-16 MiB array inside the library.  This file checks, through the C ABI, that
-its output matches heta_attention's on two calls in a row (the second call
-reuses the array the first one left behind), and that a size whose split
-scratch would not fit runs unsplit with the same result.
+16 MiB array inside the library.  This file checks, through the C ABI, on
+two calls in a row (the second call reuses the array the first one left
+behind):
+
+* where both entry points plan the same work (the split scratch fits the
+  array), that its output equals heta_attention's bit for bit;
+* where the split scratch would not fit, that it runs every dense pair
+  unsplit and still matches heta_attention within the output tolerance;
+* in both cases, that sampled rows (and every border class) match the fp64
+  oracle within the output tolerance.
 
 The file name sorts last so that a run stopping at the first failure has run
 every other test first.
@@ -17,7 +23,8 @@ import math
 import numpy as np
 import pytest
 
-from helpers import MAX_ABS, MEAN_ABS, from_dev_bf16, to_dev, to_dev_bf16
+import oracle
+from helpers import MAX_ABS, MEAN_ABS, assert_close, from_dev_bf16, sample_rows, to_dev, to_dev_bf16
 from uncertainty_routed_heterogeneous_b200 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -29,6 +36,16 @@ def _noalloc(lib):
     fn.argtypes = [vp, vp, vp] + [i] * 9 + [ctypes.c_float, vp, i, vp, vp, vp]
     fn.restype = i
     return fn
+
+
+def _against_oracle(w, q, k, v, dense_np, got, n_sample, seed):
+    """Sampled output rows (plus border classes and first/last dense rows)
+    against the fp64 oracle."""
+    rows = sample_rows(np.random.default_rng(seed), w.B, w.H, w.N, w.grid, w.win, dense_np,
+                       n_sample)
+    want = oracle.attention_rows(W.bf16_to_f32(q), W.bf16_to_f32(k), W.bf16_to_f32(v),
+                                 w.grid, w.win, dense_np, rows)
+    assert_close(got.reshape(-1, w.d)[rows], want, w.name)
 
 
 @pytest.mark.parametrize("grid,win,rho,H,d", [
@@ -62,8 +79,9 @@ def test_noalloc_matches_workspace_entry_point(gpu_lib, grid, win, rho, H, d):
         assert int(st.item()) == 0
         got = from_dev_bf16(out)
         assert np.all(np.isfinite(got)), "call %d left rows unwritten" % call
-        err = np.abs(got - want)
-        assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (call, err.max(), err.mean())
+        # the same plan and the same kernel as heta_attention: the same bits
+        assert np.array_equal(got, want), "call %d differs from heta_attention" % call
+        _against_oracle(w, q, k, v, dense.cpu().numpy(), got, 2048, call)
 
 
 def test_noalloc_runs_unsplit_when_its_array_is_too_small(gpu_lib):
@@ -97,3 +115,4 @@ def test_noalloc_runs_unsplit_when_its_array_is_too_small(gpu_lib):
     assert np.all(np.isfinite(got))
     err = np.abs(got - want)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
+    _against_oracle(w, q, k, v, dense.cpu().numpy(), got, 4096, 7)

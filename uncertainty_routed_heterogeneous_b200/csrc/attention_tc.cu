@@ -76,6 +76,7 @@ struct Params {
     // DENSE items
     int tiles_d, pairs_d, pairs_full, nsplit, n_kv_d, kv_per_split, n_dense_items;
     int max_split;    // 1: no pair is cut into key ranges (the scratch has no room)
+    int sms;          // SM count the waves of dense work are planned for
     // LOCAL items
     int box_t, box_h, box_w;
     int tiles_l, pairs_l, nbh, nbw, nkt, nkh, nkw, n_kv_l, n_local_items;
@@ -171,17 +172,17 @@ struct DPlan {
 };
 
 // The same rule as plan_attention's on the host.
-__device__ __forceinline__ DPlan dense_plan(int pairs_total, int n_kv, int max_split)
+__device__ __forceinline__ DPlan dense_plan(int pairs_total, int n_kv, int max_split, int sms)
 {
     DPlan d;
     d.pairs_total = pairs_total;
     d.pairs_full = pairs_total;
     d.nsplit = 1;
     if (pairs_total > 0 && n_kv >= 16) {
-        d.pairs_full = pairs_total / kPlanSMs * kPlanSMs;
+        d.pairs_full = pairs_total / sms * sms;
         const int rest = pairs_total - d.pairs_full;
         d.nsplit = rest > 0 ? min(max_split, n_kv / 8) : 1;
-        if (d.pairs_full > 0 && rest > kPlanSMs / 2) d.nsplit = 1;
+        if (d.pairs_full > 0 && rest > sms / 2) d.nsplit = 1;
         if (d.nsplit < 2) {  // a last wave more than half full runs whole
             d.nsplit = 1;
             d.pairs_full = pairs_total;
@@ -449,7 +450,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             sh.cpref[p.B] = acc;
             pairs_total = p.H * acc;
         }
-        sh.dplan = dense_plan(pairs_total, p.n_kv_d, p.max_split);
+        sh.dplan = dense_plan(pairs_total, p.n_kv_d, p.max_split, p.sms);
         fence_mbar_init();
         fence_proxy_async_smem();
     }
@@ -787,7 +788,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
             if (dense) {
                 const int q = tile * kTileRows + r;
                 row_valid = tile < p.tiles_d && q < it.kb;
-                if (row_valid) token = __ldg(p.dense_idx + (int64_t)it.b * p.k + q);
+                if (row_valid) {
+                    // The dense set is a subset of the sample's N tokens, listed in
+                    // increasing order (Eq. (12)-(13)).  An entry outside [0, N), or
+                    // not above the one before it, is reported and its row is
+                    // neither gathered nor stored, so no access leaves Q or out.
+                    const int32_t *dl = p.dense_idx + (int64_t)it.b * p.k;
+                    token = __ldg(dl + q);
+                    const int prev = q > 0 ? __ldg(dl + q - 1) : -1;
+                    if (token < 0 || token >= p.N || token <= prev) {
+                        raise_status(p.status, HETA_ERR_INVALID_ARG);
+                        row_valid = false;
+                        token = 0;
+                    }
+                }
                 const uint4 *src = reinterpret_cast<const uint4 *>(p.Q + (row0 + token) * D);
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
@@ -1029,10 +1043,23 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
+int plan_sms()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        sms < 1) {
+        cudaGetLastError();  // (no device visible: not an error of a later call)
+        return kDefaultSMs;
+    }
+    return sms;
+}
+
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
-                        int wh, int ww, bool per_sample_counts, bool allow_split)
+                        int wh, int ww, int sms, bool per_sample_counts, bool allow_split)
 {
     AttnPlan pl;
+    pl.sms = sms = max(sms, 1);
     pl.max_split = allow_split ? kMaxSplit : 1;
     pl.n_kv_d = (N + kTileKeys - 1) / kTileKeys;
     pl.tiles_d = (k + kTileRows - 1) / kTileRows;
@@ -1048,10 +1075,10 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
     pl.pairs_full = (int)pairs_total;
     pl.nsplit = 1;
     if (k > 0 && pl.n_kv_d >= 16) {
-        pl.pairs_full = (int)(pairs_total / kPlanSMs * kPlanSMs);
+        pl.pairs_full = (int)(pairs_total / sms * sms);
         const int64_t rest = pairs_total - pl.pairs_full;
         pl.nsplit = rest > 0 ? min(pl.max_split, pl.n_kv_d / 8) : 1;
-        if (pl.pairs_full > 0 && rest > kPlanSMs / 2) pl.nsplit = 1;
+        if (pl.pairs_full > 0 && rest > sms / 2) pl.nsplit = 1;
         if (pl.nsplit < 2) {  // a last wave more than half full runs whole
             pl.nsplit = 1;
             pl.pairs_full = (int)pairs_total;
@@ -1066,7 +1093,7 @@ AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int W
         // same way: reserve ids and scratch for the worst remainder.
         int64_t extra = 0, worst_split = 0, worst_ranges = 0;
         if (k > 0 && pl.n_kv_d >= 16) {
-            for (int rest = 1; rest < kPlanSMs && rest <= pairs_total; ++rest) {
+            for (int rest = 1; rest < sms && rest <= pairs_total; ++rest) {
                 // (the device's pairs_full may be 0, when the counts are small)
                 const int ns = min(pl.max_split, pl.n_kv_d / 8);
                 if (ns < 2) continue;
@@ -1141,6 +1168,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     p.tiles_d = pl.tiles_d; p.pairs_d = pl.pairs_d; p.pairs_full = pl.pairs_full;
     p.nsplit = pl.nsplit;
     p.max_split = pl.max_split;
+    p.sms = pl.sms;
     p.n_kv_d = pl.n_kv_d; p.kv_per_split = pl.kv_per_split; p.n_dense_items = pl.n_dense_items;
     p.box_t = pl.box_t; p.box_h = pl.box_h; p.box_w = pl.box_w;
     p.tiles_l = pl.tiles_l; p.pairs_l = pl.pairs_l; p.nbh = pl.nbh; p.nbw = pl.nbw;
@@ -1163,10 +1191,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
 
     cudaError_t e = cudaMemsetAsync(workspace, 0, pl.zero_bytes, s);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = kPlanSMs;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int grid = min(pl.total_items, sms);
+    const int grid = min(pl.total_items, pl.sms);
     if (D == 64) {
         e = cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Cfg<64>::kSmem);

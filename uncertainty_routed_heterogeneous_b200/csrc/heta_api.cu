@@ -48,7 +48,7 @@ heta_status heta_route(const float *u, int B, int N, int k, int32_t *dense_idx,
 {
     if (B < 1 || N < 1 || k < 0 || k > N) return HETA_ERR_INVALID_ARG;
     if ((int64_t)B * N >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
-    if (N > heta::kRouteMaxN) return HETA_ERR_UNSUPPORTED;
+    if (N > heta::kRouteClusterMaxN) return HETA_ERR_UNSUPPORTED;
     if (!u || (k > 0 && !dense_idx) || (k < N && !local_idx)) return HETA_ERR_INVALID_ARG;
     if (!aligned16(u) || (dense_idx && !aligned16(dense_idx)) ||
         (local_idx && !aligned16(local_idx)) || (thresh_out && !aligned16(thresh_out)) ||
@@ -106,7 +106,7 @@ heta_status heta_route_threshold(const float *u, int B, int N, double c, int32_t
 {
     if (B < 1 || N < 1 || !std::isfinite(c)) return HETA_ERR_INVALID_ARG;
     if ((int64_t)B * N >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
-    if (N > heta::kRouteMaxN) return HETA_ERR_UNSUPPORTED;
+    if (N > heta::kRouteClusterMaxN) return HETA_ERR_UNSUPPORTED;
     if (!u || !counts || !dense_idx || !local_idx) return HETA_ERR_INVALID_ARG;
     if (!aligned16(u) || !aligned16(counts) || !aligned16(dense_idx) || !aligned16(local_idx) ||
         (thresh_out && !aligned16(thresh_out)) || (mask_out && !aligned16(mask_out)))
@@ -153,7 +153,7 @@ int attention_checked(const uint16_t *Q, const uint16_t *K, const uint16_t *V, i
         (dense_idx && !aligned16(dense_idx)) || !aligned16(workspace))
         return HETA_ERR_INVALID_ARG;
     const AttnPlan plan =
-        plan_attention(B, H, d, N, k, Tg, Hg, Wg, wt, wh, ww, false, allow_split);
+        plan_attention(B, H, d, N, k, Tg, Hg, Wg, wt, wh, ww, plan_sms(), false, allow_split);
     if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
     AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;
@@ -174,7 +174,8 @@ heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, int Hg, i
     if (!bytes) return HETA_ERR_INVALID_ARG;
     const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k);
     if (st != HETA_OK) return st;
-    *bytes = heta::plan_attention(B, H, d, Tg * Hg * Wg, k, Tg, Hg, Wg, wt, wh, ww)
+    *bytes = heta::plan_attention(B, H, d, Tg * Hg * Wg, k, Tg, Hg, Wg, wt, wh, ww,
+                                  heta::plan_sms())
                  .workspace_bytes;
     return HETA_OK;
 }
@@ -187,7 +188,8 @@ heta_status heta_attention_counts_workspace_size(int B, int H, int d, int Tg, in
     const heta_status st = check_attention_shape(B, H, d, Tg, Hg, Wg, wt, wh, ww, k_cap);
     if (st != HETA_OK) return st;
     if (B > heta::kMaxCountsSamples) return HETA_ERR_UNSUPPORTED;
-    *bytes = heta::plan_attention(B, H, d, Tg * Hg * Wg, k_cap, Tg, Hg, Wg, wt, wh, ww, true)
+    *bytes = heta::plan_attention(B, H, d, Tg * Hg * Wg, k_cap, Tg, Hg, Wg, wt, wh, ww,
+                                  heta::plan_sms(), true)
                  .workspace_bytes;
     return HETA_OK;
 }
@@ -222,7 +224,7 @@ heta_status heta_attention_counts(const uint16_t *Q, const uint16_t *K, const ui
         !aligned16(counts) || (dense_idx && !aligned16(dense_idx)) || !aligned16(workspace))
         return HETA_ERR_INVALID_ARG;
     const heta::AttnPlan plan =
-        heta::plan_attention(B, H, d, N, k_cap, Tg, Hg, Wg, wt, wh, ww, true);
+        heta::plan_attention(B, H, d, N, k_cap, Tg, Hg, Wg, wt, wh, ww, heta::plan_sms(), true);
     if (workspace_bytes < plan.workspace_bytes) return HETA_ERR_INVALID_ARG;
     heta::AttnArgs a;
     a.Q = Q; a.K = K; a.V = V; a.out = out; a.dense_idx = dense_idx; a.status = status_dev;

@@ -17,6 +17,10 @@ __device__ __forceinline__ void raise_status(int32_t *status, int32_t code)
 
 // Largest N one routing CTA can hold in shared memory (4 bytes per token).
 constexpr int kRouteMaxN = 53248;
+// Largest N the routing calls take: a cluster of eight CTAs holds one eighth
+// of a sample each, up to 49152 tokens (192 KB) a CTA.  Samples above
+// kRouteMaxN always take the cluster kernels, whatever the batch size.
+constexpr int kRouteClusterMaxN = 8 * 49152;
 
 cudaError_t launch_route(const float *u, int B, int N, int k, int32_t *dense_idx,
                          int32_t *local_idx, float *thresh, uint8_t *mask,
@@ -56,6 +60,7 @@ struct AttnArgs {
 
 // How one heta_attention call is cut into work items, and its workspace.
 struct AttnPlan {
+    int sms;                  // SMs the waves of dense work are planned for (the grid size)
     int tiles_d, pairs_d, n_kv_d, pairs_full, nsplit, kv_per_split, n_dense_items;
     int max_split;            // most key ranges a dense pair may be cut into
     int box_t, box_h, box_w;  // LOCAL query box (box_t * box_h * box_w == 128)
@@ -64,9 +69,11 @@ struct AttnPlan {
     size_t off_fix, off_ml, off_o, zero_bytes, workspace_bytes;
 };
 
-// SM count the work split is planned for (B200).  Only the balance depends
-// on it, never the result; the launch itself uses the device's real count.
-constexpr int kPlanSMs = 148;
+// The current device's multiprocessor count, which the dense work is cut into
+// waves for (only the balance and the scratch size depend on it, never the
+// result); kDefaultSMs (a B200) when no device is visible.
+constexpr int kDefaultSMs = 148;
+int plan_sms();
 
 // Samples heta_attention_counts takes (its per-sample pair prefix lives in
 // shared memory).
@@ -77,7 +84,7 @@ constexpr int kMaxCountsSamples = 1024;
 // allow_split = false runs every dense pair over its whole key range, so the
 // workspace is only the work counter.
 AttnPlan plan_attention(int B, int H, int d, int N, int k, int Tg, int Hg, int Wg, int wt,
-                        int wh, int ww, bool per_sample_counts = false,
+                        int wh, int ww, int sms, bool per_sample_counts = false,
                         bool allow_split = true);
 
 // heta_attention's body once its shape is checked, with the split choice open

@@ -1,11 +1,13 @@
-// route_cluster.cu -- per-sample top-k routing for a few samples: one sample
-// over a cluster of eight CTAs.
+// route_cluster.cu -- per-sample top-k routing for a few samples, or for
+// samples too large for one SM's shared memory: one sample over a cluster of
+// eight CTAs.
 //
 // "Where Compute Matters: Heterogeneous Attention for Efficient Video
 // Diffusion", §3.2.2 Eq. (11)-(12), in top-k form (k = ceil(rho*N) per
 // sample, equal u taken in increasing token index, -0.0 == +0.0): the same
 // selection as route.cu, whose one CTA a sample leaves a single-sample call
-// latency-bound on one SM.  Here the sample's quads are cut into eight
+// latency-bound on one SM and holds at most kRouteMaxN tokens (a 720p Wan
+// latent, 21x45x80 = 75600 tokens, needs two SMs' worth).  Here the sample's quads are cut into eight
 // contiguous slices, one a CTA, and the CTAs combine what they found through
 // distributed shared memory:
 //   1. each CTA loads its slice and its min / max; the cluster's min / max;
@@ -518,8 +520,7 @@ route_cluster_kernel(const float *__restrict__ u, int N, int k,
 
 bool route_cluster_fits(int B, int N)
 {
-    (void)N;
-    return B >= 1 && B <= kRouteClusterMaxB;
+    return B >= 1 && N <= kRouteClusterMaxN && (B <= kRouteClusterMaxB || N > kRouteMaxN);
 }
 
 cudaError_t launch_route_cluster(const float *u, int B, int N, int k, int32_t *dense_idx,
@@ -529,7 +530,7 @@ cudaError_t launch_route_cluster(const float *u, int B, int N, int k, int32_t *d
     // a slice: up to ceil(quads / 8) quads
     const int nq = (N + 3 + 3) / 4;
     const size_t smem = sizeof(uint4) * (size_t)((nq + kCl - 1) / kCl);
-    const int max_smem = (int)(sizeof(uint4) * ((kRouteMaxN / 4 + 2 + kCl - 1) / kCl));
+    const int max_smem = (int)(sizeof(uint4) * ((kRouteClusterMaxN / 4 + 2 + kCl - 1) / kCl));
     auto kern = mask ? route_cluster_kernel<true> : route_cluster_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          max_smem);

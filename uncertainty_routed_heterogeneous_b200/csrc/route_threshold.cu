@@ -9,9 +9,10 @@
 // into eight slices of ceil(N/8) tokens; in each slice thread t (of 1024)
 // adds its tokens t, t+1024, ... in fp64, a shuffle tree sums each warp and
 // a second tree the 32 warps; the eight slice sums are added in slice order.
-// Up to eight samples a call, the slices are the eight CTAs of a cluster
-// (their sums and dense counts exchanged through distributed shared memory);
-// otherwise one CTA per sample computes the same eight slice sums.  Either
+// Up to eight samples a call, and for samples too large for one CTA's
+// shared memory, the slices are the eight CTAs of a cluster (their sums and
+// dense counts exchanged through distributed shared memory); otherwise one
+// CTA per sample computes the same eight slice sums.  Either
 // way the same T comes out of the same u.  Every u is compared with T in
 // fp64; warp ballots compact both index lists in increasing order.
 #include "heta_internal.cuh"
@@ -351,9 +352,9 @@ cudaError_t launch_route_threshold(const float *u, int B, int N, double c, int32
                                    int32_t *dense_idx, int32_t *local_idx, double *thresh,
                                    uint8_t *mask, int32_t *status, cudaStream_t s)
 {
-    if (B <= kRouteClusterMaxB) {
+    if (B <= kRouteClusterMaxB || N > kRouteMaxN) {
         const int L = (N + kSlices - 1) / kSlices;
-        const int Lmax = (kRouteMaxN + kSlices - 1) / kSlices;
+        const int Lmax = (kRouteClusterMaxN + kSlices - 1) / kSlices;
         cudaError_t e = cudaFuncSetAttribute(route_threshold_cluster_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)(sizeof(float) * Lmax));

@@ -1,10 +1,19 @@
 """Host-side plumbing for running the path on several GPUs of one node.
 
-The routed-attention step shards without any data exchange: samples (and,
-inside a sample, heads) are independent, and routing is per sample.  Each
-rank therefore runs whole steps on its own samples and the ranks meet only at
-the barriers around the timed region and in one max-reduction of the elapsed
-time.  Nothing here touches the data path.
+Two ways to shard the routed-attention step:
+
+* samples (the default): samples are independent and routing is per sample,
+  so each rank runs whole steps on its own samples and the ranks meet only at
+  the barriers around the timed region and in one max-reduction of the
+  elapsed time (weak scaling, no data-path collective);
+* heads of one sample: attention heads are independent (Eq. (2)-(3) act per
+  head), so rank r takes the contiguous head block ``head_range(H, G, r)``
+  of Q/K/V and routes the sample's full u itself (routing is deterministic,
+  so every rank gets the same lists); the uncertainty head's token rows are
+  split the same way, and its output -- which every rank needs to route the
+  next step -- is the one real exchange, an all-gather of equal slices
+  (``all_gather_equal``), as is the optional all-gather of the output along
+  heads.
 """
 import dataclasses
 import os
@@ -56,6 +65,25 @@ def head_range(H: int, world: int, rank: int):
     base, extra = divmod(H, world)
     lo = rank * base + min(rank, extra)
     return lo, lo + base + (1 if rank < extra else 0)
+
+
+def row_range(n: int, world: int, rank: int):
+    """Contiguous block [lo, hi) of n rows (tokens) for rank `rank`; equal blocks
+    when world divides n (what ``all_gather_equal`` needs)."""
+    return head_range(n, world, rank)
+
+
+def all_gather_equal(local, info: RankInfo):
+    """The ranks' equal-sized tensors concatenated in rank order, as one flat
+    tensor on local's device (local itself, flattened, for one rank)."""
+    if info.world == 1:
+        return local.reshape(-1)
+    import torch
+    import torch.distributed as dist
+    flat = local.contiguous().reshape(-1)
+    out = torch.empty(info.world * flat.numel(), dtype=flat.dtype, device=flat.device)
+    dist.all_gather_into_tensor(out, flat)
+    return out
 
 
 def max_over_ranks(x: float, info: RankInfo, device=None) -> float:

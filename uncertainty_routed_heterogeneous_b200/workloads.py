@@ -61,6 +61,12 @@ SWEEP_RHOS = (0.05, 0.1, 0.2, 0.35, 0.5)
 BATCHED = Workload("wan2.1-1.3b-batched-b2", B=2, H=12, d=128,
                    grid=(21, 30, 52), win=(3, 9, 9), rho=0.2, u_kind="smooth",
                    qkv_seed=1, u_seeds=(5, 6), C=1536)
+# The Wan2.1-1.3B layer at 720p (81 frames -> 21 latent frames, 720x1280 ->
+# 45x80 after the 16x spatial compression and 2x2 patchify): N = 75600, the
+# resolution at which the paper puts self-attention at 82% of compute.
+WAN21_720P = Workload("wan2.1-1.3b-720p-21x45x80", B=1, H=12, d=128,
+                      grid=(21, 45, 80), win=(3, 9, 9), rho=0.2, u_kind="smooth",
+                      qkv_seed=1, u_seeds=(2,), C=1536)
 
 
 def sweep(rho: float, u_kind: str) -> Workload:
@@ -70,7 +76,7 @@ def sweep(rho: float, u_kind: str) -> Workload:
                    rho=rho, u_kind=u_kind, u_seeds=(7,))
 
 
-ALL = {w.name: w for w in (TINY, WAN21, WAN22, BATCHED)}
+ALL = {w.name: w for w in (TINY, WAN21, WAN22, BATCHED, WAN21_720P)}
 
 # the window sizes the paper's window ablation compares (its default 11^3,
 # plus 9^3 and 13^3), at the Wan2.1 latent shape
