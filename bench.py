@@ -70,6 +70,9 @@ def parse_args():
                    help="mark route / attention / head of every step with NVTX ranges")
     p.add_argument("--cpu-seconds", type=float, default=10.0,
                    help="minimum host time the cpu_baseline oracle sample runs for")
+    p.add_argument("--no-flex-compare", action="store_true",
+                   help="skip timing PyTorch FlexAttention on the same mask (the paper's own "
+                        "latency instrument; a comparison point, not part of the product)")
     p.add_argument("--shard", choices=["samples", "heads"], default="samples",
                    help="samples: each rank runs its own sample (weak scaling, the default); "
                         "heads: the ranks split one sample's heads and the head's token rows "
@@ -434,6 +437,79 @@ def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
     return res
 
 
+def flex_compare(heta, torch, dev, w, d_Q, d_K, d_V, dense, local, ours, ours_ms):
+    """The same heterogeneous mask realised with PyTorch FlexAttention, the
+    paper's latency instrument (Where Compute Matters, §4 "Compute Complexity
+    Assessment"; Table 5 counts the BlockMask construction in).  A comparison
+    point only: the query rows are permuted so the dense ones come first (the
+    dense query blocks then attend to every key block and the local ones to the
+    key blocks their windows reach), the block mask is built from the routing,
+    flex_attention runs the compiled block-sparse kernel, and the rows are put
+    back in token order.  Returns times, the speedup of our kernel and the
+    largest difference between the two outputs on the same inputs."""
+    import time as _time
+
+    from torch.nn.attention.flex_attention import create_block_mask, flex_attention
+    Tg, Hg, Wg = w.grid
+    wt, wh, ww = w.win
+    HW = Hg * Wg
+    k = dense.shape[1]
+    perm = torch.cat([dense[0], local[0]]).to(torch.int64)
+
+    def mask_mod(b, h, q_idx, kv_idx):
+        tok = perm[q_idx]
+        t, hh, x = tok // HW, (tok // Wg) % Hg, tok % Wg
+        tk, hk, xk = kv_idx // HW, (kv_idx // Wg) % Hg, kv_idx % Wg
+        st = torch.clamp(t - wt // 2, 0, Tg - wt)
+        sh = torch.clamp(hh - wh // 2, 0, Hg - wh)
+        sx = torch.clamp(x - ww // 2, 0, Wg - ww)
+        inwin = ((tk >= st) & (tk < st + wt) & (hk >= sh) & (hk < sh + wh) &
+                 (xk >= sx) & (xk < sx + ww))
+        return (q_idx < k) | inwin
+
+    flex = torch.compile(flex_attention, dynamic=False)
+    make_mask = torch.compile(create_block_mask)
+    t0 = _time.perf_counter()
+    bm = make_mask(mask_mod, 1, None, w.N, w.N, device=dev)
+    Qp = d_Q.index_select(2, perm)
+    res = flex(Qp, d_K, d_V, block_mask=bm)
+    out = torch.empty_like(d_Q)
+    out.index_copy_(2, perm, res)
+    torch.cuda.synchronize()
+    compile_s = _time.perf_counter() - t0
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    mask_ms = timed(lambda: make_mask(mask_mod, 1, None, w.N, w.N, device=dev))
+    attn_ms = timed(lambda: flex(Qp, d_K, d_V, block_mask=bm))
+
+    def whole():
+        b2 = make_mask(mask_mod, 1, None, w.N, w.N, device=dev)
+        r = flex(d_Q.index_select(2, perm), d_K, d_V, block_mask=b2)
+        out.index_copy_(2, perm, r)
+    total_ms = timed(whole)
+    diff = float((out.float() - ours.float()).abs().max())
+    fl = heta.attention_flops(w.B, w.H, w.d, w.N, k, w.M)
+    return {"what": "torch FlexAttention (compiled, block size 128) on the same mask, query "
+                    "rows permuted dense-first; a comparison point, not the product",
+            "blockmask_ms": mask_ms, "flex_attention_ms": attn_ms,
+            "total_ms_with_blockmask_and_permutation": total_ms,
+            "algorithmic_tflops_of_flex": fl / (attn_ms * 1e9),
+            "ours_attention_ms": ours_ms, "speedup_ours_vs_flex_total": total_ms / ours_ms,
+            "speedup_ours_vs_flex_kernel": attn_ms / ours_ms,
+            "max_abs_diff_vs_ours": diff, "first_call_s": compile_s,
+            "sparsity_of_blockmask": float(bm.sparsity()) if hasattr(bm, "sparsity") else None}
+
+
 def run_heta(args, info):
     import torch
 
@@ -528,6 +604,17 @@ def run_heta(args, info):
     # the last timed step's routing and output, checked against the oracle
     # once all timing is done
     timed = (dense.cpu(), local.cpu(), out.cpu())
+
+    # ---- the same mask through PyTorch FlexAttention (comparison point) -------
+    flex = None
+    if not args.no_flex_compare and info.rank == 0:
+        try:
+            heta.attention(d_Q, d_K, d_V, w.grid, w.win, dense, out=out, workspace=ws)
+            torch.cuda.synchronize()
+            flex = flex_compare(heta, torch, dev, w, d_Q, d_K, d_V, dense, local, out, attn_ms)
+        except Exception as e:  # noqa: BLE001 -- a comparison leg never fails the bench
+            flex = {"unavailable": "%s: %s" % (type(e).__name__, str(e)[:300])}
+        torch.cuda.synchronize()
 
     # ---- our own full dense attention (rho = 1) at the same shape -----------
     dense_cmp = None
@@ -786,6 +873,7 @@ def run_heta(args, info):
                           (head_ms * 1e6),
                           "peak": peaks["hbm_gbs"], "unit": "GB/s"},
         "dense_compare": dense_cmp,
+        "flex_compare": flex,
         "window_sweep": win_sweep,
         "other_configs": others,
         "threshold_mode": thr,
