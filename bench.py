@@ -437,6 +437,29 @@ def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
     return res
 
 
+def flex_mask_mod(torch, perm, k, grid, win):
+    """FlexAttention mask of the heterogeneous attention with the query rows
+    permuted dense-first (perm = dense ids, then local ids): query position q
+    attends to every key when q < k, else to the keys of the clamped window of
+    its token perm[q] (start = clamp(p - w // 2, 0, extent - w) per axis)."""
+    Tg, Hg, Wg = grid
+    wt, wh, ww = win
+    HW = Hg * Wg
+
+    def mask_mod(b, h, q_idx, kv_idx):
+        tok = perm[q_idx]
+        t, hh, x = tok // HW, (tok // Wg) % Hg, tok % Wg
+        tk, hk, xk = kv_idx // HW, (kv_idx // Wg) % Hg, kv_idx % Wg
+        st = torch.clamp(t - wt // 2, 0, Tg - wt)
+        sh = torch.clamp(hh - wh // 2, 0, Hg - wh)
+        sx = torch.clamp(x - ww // 2, 0, Wg - ww)
+        inwin = ((tk >= st) & (tk < st + wt) & (hk >= sh) & (hk < sh + wh) &
+                 (xk >= sx) & (xk < sx + ww))
+        return (q_idx < k) | inwin
+
+    return mask_mod
+
+
 def flex_compare(heta, torch, dev, w, d_Q, d_K, d_V, dense, local, ours, ours_ms):
     """The same heterogeneous mask realised with PyTorch FlexAttention, the
     paper's latency instrument (Where Compute Matters, §4 "Compute Complexity
@@ -450,23 +473,9 @@ def flex_compare(heta, torch, dev, w, d_Q, d_K, d_V, dense, local, ours, ours_ms
     import time as _time
 
     from torch.nn.attention.flex_attention import create_block_mask, flex_attention
-    Tg, Hg, Wg = w.grid
-    wt, wh, ww = w.win
-    HW = Hg * Wg
     k = dense.shape[1]
     perm = torch.cat([dense[0], local[0]]).to(torch.int64)
-
-    def mask_mod(b, h, q_idx, kv_idx):
-        tok = perm[q_idx]
-        t, hh, x = tok // HW, (tok // Wg) % Hg, tok % Wg
-        tk, hk, xk = kv_idx // HW, (kv_idx // Wg) % Hg, kv_idx % Wg
-        st = torch.clamp(t - wt // 2, 0, Tg - wt)
-        sh = torch.clamp(hh - wh // 2, 0, Hg - wh)
-        sx = torch.clamp(x - ww // 2, 0, Wg - ww)
-        inwin = ((tk >= st) & (tk < st + wt) & (hk >= sh) & (hk < sh + wh) &
-                 (xk >= sx) & (xk < sx + ww))
-        return (q_idx < k) | inwin
-
+    mask_mod = flex_mask_mod(torch, perm, k, w.grid, w.win)
     flex = torch.compile(flex_attention, dynamic=False)
     make_mask = torch.compile(create_block_mask)
     t0 = _time.perf_counter()

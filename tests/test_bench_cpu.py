@@ -75,3 +75,30 @@ def test_reference_line_under_torchrun_comes_from_rank_0_only():
     assert len(lines) == 1
     assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
     assert lines[0]["config"]["workload"] == W.TINY.name
+
+
+def test_flex_comparison_mask_is_the_oracles_mask():
+    """The FlexAttention comparison in bench.py realises the same mask: run
+    eagerly on CPU on a tiny grid (dense query rows first, as bench.py
+    permutes them), put back in token order, it equals the fp64 oracle."""
+    import numpy as np
+    import torch
+    from torch.nn.attention.flex_attention import create_block_mask, flex_attention
+
+    import oracle
+    sys.path.insert(0, ROOT)
+    import bench
+    w = W.scaled(W.WAN21, H=2, d=64, grid=(4, 6, 10), win=(3, 3, 5), u_kind="uniform",
+                 u_seeds=(13,))
+    q, k, v = (W.bf16_to_f32(a) for a in W.make_qkv(w))
+    kk = oracle.dense_count(w.N, w.rho)
+    dense, local, _ = oracle.route(W.make_u(w), kk)
+    perm = torch.from_numpy(np.concatenate([dense[0], local[0]]).astype(np.int64))
+    mask_mod = bench.flex_mask_mod(torch, perm, kk, w.grid, w.win)
+    bm = create_block_mask(mask_mod, 1, None, w.N, w.N, device="cpu", BLOCK_SIZE=16)
+    Q, K, V = (torch.from_numpy(a).double() for a in (q, k, v))
+    res = flex_attention(Q.index_select(2, perm), K, V, block_mask=bm)
+    out = torch.empty_like(Q)
+    out.index_copy_(2, perm, res)
+    want = oracle.attention(q, k, v, w.grid, w.win, dense)
+    assert np.abs(out.numpy() - want).max() < 1e-9
