@@ -120,9 +120,10 @@ HETA_API heta_status heta_route(const float *u, int B, int N, int k,
  *   local_out  [B,N-k] int32 out: the complements, increasing.
  *   mask_out   [B,N] uint8 out, or NULL: m_i of the new sets, 1 = local.
  *
- * Requires 0 <= s <= min(k, N-k), block >= 0, N <= 53248 (one sample in
- * one SM's shared memory) and B*N < 2^31; pointers 16-byte aligned.  One CTA
- * per sample.
+ * Requires 0 <= s <= min(k, N-k), block >= 0, N <= 393216 and B*N < 2^31;
+ * pointers 16-byte aligned.  One CTA per sample: up to N = 53248 its draws
+ * are kept in shared memory, above that (a 720p latent has 75600 tokens)
+ * each pass computes them again.
  */
 HETA_API heta_status heta_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
                                      uint64_t seed, int block, int32_t *dense_out,

@@ -152,7 +152,7 @@ def test_swap_entry_point_validates_on_the_host(lib):
     big_s[3], big_s[4] = 90, 11  # s > N - k
     assert sw(*big_s) == heta.HETA_ERR_INVALID_ARG
     too_big = list(ok)
-    too_big[2], too_big[3], too_big[4] = 60000, 20, 5
+    too_big[2], too_big[3], too_big[4] = 8 * 49152 + 1, 20, 5
     assert sw(*too_big) == heta.HETA_ERR_UNSUPPORTED
     no_local = list(ok)
     no_local[8] = N

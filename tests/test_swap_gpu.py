@@ -51,7 +51,9 @@ def test_swap_wan21_table8_setting(gpu_lib, block):
 
 
 @pytest.mark.parametrize("N,k,s", [(1001, 300, 77), (4099, 2049, 2050), (53248, 10650, 3728),
-                                   (64, 32, 32), (300, 150, 0), (257, 1, 1)])
+                                   (64, 32, 32), (300, 150, 0), (257, 1, 1),
+                                   # above one SM's shared memory: draws computed per pass
+                                   (53249, 10650, 3728), (75600, 15120, 5292)])
 def test_swap_sizes(gpu_lib, N, k, s):
     rng = np.random.default_rng(N)
     u = rng.standard_normal((3, N)).astype(np.float32)
@@ -74,7 +76,8 @@ def test_swap_bad_index_is_reported(gpu_lib):
     assert int(st.item()) == heta.HETA_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("N,k,s,B", [(32760, 6552, 2294, 2), (1001, 300, 77, 3)])
+@pytest.mark.parametrize("N,k,s,B", [(32760, 6552, 2294, 2), (1001, 300, 77, 3),
+                                     (75600, 15120, 5292, 1)])
 def test_swap_blocks_matches_one_block_calls(gpu_lib, N, k, s, B):
     """All 30 blocks of a step in one launch (heta_route_swap_blocks) give,
     block for block, the lists of 30 single-block calls; blocks 0 and 29 are

@@ -73,7 +73,7 @@ heta_status heta_route_swap_blocks(const int32_t *dense_idx, int B, int N, int k
     if ((int64_t)block0 + nblocks - 1 > INT32_MAX) return HETA_ERR_INVALID_ARG;
     if ((int64_t)B * N * nblocks >= (int64_t)1 << 31) return HETA_ERR_INVALID_ARG;
     if ((int64_t)B * nblocks > INT32_MAX) return HETA_ERR_INVALID_ARG;
-    if (N > heta::kRouteMaxN) return HETA_ERR_UNSUPPORTED;
+    if (N > heta::kRouteClusterMaxN) return HETA_ERR_UNSUPPORTED;
     if ((k > 0 && (!dense_idx || !dense_out)) || (k < N && !local_out))
         return HETA_ERR_INVALID_ARG;
     if ((dense_idx && !aligned16(dense_idx)) || (dense_out && !aligned16(dense_out)) ||

@@ -14,7 +14,9 @@
 // draws are computed once into shared memory, each set's s smallest draws
 // are found by the same three-pass radix select as the top-k routing (on the
 // complemented draws, so "largest" means smallest), and a ballot compaction
-// writes both new lists in increasing order.
+// writes both new lists in increasing order.  A sample too large for its
+// draws to fit in shared memory (N > kRouteMaxN, e.g. a 720p latent) keeps
+// only the bitmap there and computes each token's draw again in every pass.
 #include "heta_internal.cuh"
 #include "radix_select.cuh"
 
@@ -46,6 +48,7 @@ __device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint3
     return c0;
 }
 
+template <bool kStored>
 __global__ void __launch_bounds__(kThreads, 1)
 route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t seed_lo,
                   uint32_t seed_hi, int block0, int32_t *dense_out, int32_t *local_out,
@@ -57,8 +60,8 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
     const int beta = blockIdx.x / B;
     const int block = block0 + beta;
     extern __shared__ uint32_t dyn[];
-    uint32_t *key = dyn;       // [N] complemented draws: larger key = smaller draw
-    uint32_t *bits = dyn + N;  // [ceil(N/32)] dense set of the input routing
+    uint32_t *key = dyn;                    // [N] complemented draws (kStored)
+    uint32_t *bits = kStored ? dyn + N : dyn;  // [ceil(N/32)] dense set of the input routing
     __shared__ uint32_t hist[2048];  // radix digits; or [group][1024] top-10-bit buckets
     __shared__ uint32_t cand_k[2][kSwapCand];
     __shared__ int cand_i[2][kSwapCand];
@@ -100,13 +103,17 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
     auto in_group = [&](int i, int g) -> bool {
         return (int)((bits[i >> 5] >> (i & 31)) & 1u) == g;
     };
+    // token i's complemented draw: larger key = smaller draw
+    auto draw = [&](int i) -> uint32_t {
+        return ~philox_word0((uint32_t)i, (uint32_t)b, (uint32_t)block, 0u, seed_lo, seed_hi);
+    };
+    auto key_of = [&](int i) -> uint32_t { return kStored ? key[i] : draw(i); };
 
     // ---- 2. the draws, with each group's histogram of their top 10 bits
     // (group 0: the input's local set, 1: its dense set)
     for (int i = tid; i < N; i += kThreads) {
-        const uint32_t kk =
-            ~philox_word0((uint32_t)i, (uint32_t)b, (uint32_t)block, 0u, seed_lo, seed_hi);
-        key[i] = kk;
+        const uint32_t kk = draw(i);
+        if (kStored) key[i] = kk;
         atomicAdd(&hist[(in_group(i, 1) ? 1024 : 0) + (kk >> 22)], 1u);
     }
     __syncthreads();
@@ -141,7 +148,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
         // the tokens of each group in buckets above it: those all change sets
         uint32_t above[2] = {0u, 0u};
         for (int i = seg_lo + lane; i < seg_hi; i += 32) {
-            const uint32_t kk = key[i];
+            const uint32_t kk = key_of(i);
             const int g = in_group(i, 1) ? 1 : 0;
             const uint32_t bk = kk >> 22;
             above[g] += bk > bkt[g];
@@ -189,14 +196,14 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
         for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
         __syncthreads();
         for (int i = tid; i < N; i += kThreads)
-            if (in_group(i, g)) atomicAdd(&hist[key[i] >> 21], 1u);
+            if (in_group(i, g)) atomicAdd(&hist[key_of(i) >> 21], 1u);
         __syncthreads();
         find_digit<kThreads>(hist, 2048, (uint32_t)s, warp_tot, &s_digit, &s_rank);
         const uint32_t d1 = s_digit, r1 = s_rank;
         for (int i = tid; i < 2048; i += kThreads) hist[i] = 0u;
         __syncthreads();
         for (int i = tid; i < N; i += kThreads) {
-            const uint32_t kk = key[i];
+            const uint32_t kk = key_of(i);
             if ((kk >> 21) == d1 && in_group(i, g)) atomicAdd(&hist[(kk >> 10) & 2047u], 1u);
         }
         __syncthreads();
@@ -205,7 +212,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
         for (int i = tid; i < 1024; i += kThreads) hist[i] = 0u;
         __syncthreads();
         for (int i = tid; i < N; i += kThreads) {
-            const uint32_t kk = key[i];
+            const uint32_t kk = key_of(i);
             if ((kk >> 10) == p2 && in_group(i, g)) atomicAdd(&hist[kk & 1023u], 1u);
         }
         __syncthreads();
@@ -255,7 +262,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
             const int i = base + lane;
             const bool valid = i < seg_hi;
             const int g = valid && in_group(i, 1) ? 1 : 0;
-            const bool dense = valid && ((g == 1) != changes(valid ? key[i] : 0u, i, g));
+            const bool dense = valid && ((g == 1) != changes(valid ? key_of(i) : 0u, i, g));
             const unsigned d_mask = __ballot_sync(0xffffffffu, dense);
             const uint32_t pos = rd + __popc(d_mask & lt);
             // the swap keeps |dense| == k; the bounds only guard memory
@@ -274,7 +281,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
         if (s > 0) {
             for (int i = seg_lo + lane; i < seg_hi; i += 32) {
                 const int g = in_group(i, 1) ? 1 : 0;
-                n_eq[g] += key[i] == kth[g];
+                n_eq[g] += key_of(i) == kth[g];
             }
         }
     #pragma unroll
@@ -301,7 +308,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
 
         // new dense flag of token i (eq_rank: its rank among its group's keys equal to K)
         auto selected = [&](int i, int g, uint32_t eq_rank) -> bool {
-            const uint32_t kk = key[i];
+            const uint32_t kk = key_of(i);
             return s > 0 && (kk > kth[g] || (kk == kth[g] && eq_rank < take[g]));
         };
 
@@ -313,7 +320,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
                 const int i = base + lane;
                 const bool valid = i < seg_hi;
                 const int g = valid && in_group(i, 1) ? 1 : 0;
-                const bool eq = valid && key[i] == kth[g];
+                const bool eq = valid && key_of(i) == kth[g];
                 const unsigned eq0 = __ballot_sync(0xffffffffu, eq && g == 0);
                 const unsigned eq1 = __ballot_sync(0xffffffffu, eq && g == 1);
                 const uint32_t rank = g ? re[1] + __popc(eq1 & lt) : re[0] + __popc(eq0 & lt);
@@ -345,7 +352,7 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
             const int i = base + lane;
             const bool valid = i < seg_hi;
             const int g = valid && in_group(i, 1) ? 1 : 0;
-            const bool eq = valid && key[i] == kth[g];
+            const bool eq = valid && key_of(i) == kth[g];
             const unsigned eq0 = __ballot_sync(0xffffffffu, eq && g == 0);
             const unsigned eq1 = __ballot_sync(0xffffffffu, eq && g == 1);
             const uint32_t rank = g ? re[1] + __popc(eq1 & lt) : re[0] + __popc(eq0 & lt);
@@ -370,7 +377,8 @@ route_swap_kernel(const int32_t *dense_idx, int B, int N, int k, int s, uint32_t
 
 size_t route_swap_smem_bytes(int N)
 {
-    return sizeof(uint32_t) * ((size_t)N + (size_t)((N + 31) / 32));
+    const size_t words = (size_t)((N + 31) / 32);  // the bitmap
+    return sizeof(uint32_t) * (N <= kRouteMaxN ? (size_t)N + words : words);
 }
 
 cudaError_t launch_route_swap(const int32_t *dense_idx, int B, int N, int k, int s,
@@ -378,13 +386,15 @@ cudaError_t launch_route_swap(const int32_t *dense_idx, int B, int N, int k, int
                               int32_t *local_out, uint8_t *mask, int32_t *status,
                               cudaStream_t st)
 {
-    cudaError_t e = cudaFuncSetAttribute(route_swap_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)route_swap_smem_bytes(kRouteMaxN));
+    const bool stored = N <= kRouteMaxN;
+    auto kern = stored ? route_swap_kernel<true> : route_swap_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (int)(stored ? route_swap_smem_bytes(kRouteMaxN) : route_swap_smem_bytes(kRouteClusterMaxN)));
     if (e != cudaSuccess) return e;
-    route_swap_kernel<<<(unsigned)((int64_t)B * nblocks), kThreads, route_swap_smem_bytes(N),
-                        st>>>(dense_idx, B, N, k, s, (uint32_t)seed, (uint32_t)(seed >> 32),
-                              block0, dense_out, local_out, mask, status);
+    kern<<<(unsigned)((int64_t)B * nblocks), kThreads, route_swap_smem_bytes(N), st>>>(
+        dense_idx, B, N, k, s, (uint32_t)seed, (uint32_t)(seed >> 32), block0, dense_out,
+        local_out, mask, status);
     return cudaGetLastError();
 }
 
