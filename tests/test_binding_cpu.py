@@ -26,6 +26,8 @@ CALLS = {
                                                         N, 1, 7, 0, 2),
     "attention": lambda: heta.attention(*_qkv(), GRID, WIN,
                                         torch.zeros((1, 4), dtype=torch.int32)),
+    "attention_noalloc": lambda: heta.attention_noalloc(*_qkv(), GRID, WIN,
+                                                        torch.zeros((1, 4), dtype=torch.int32)),
     "attention_counts": lambda: heta.attention_counts(*_qkv(), GRID, WIN,
                                                       torch.zeros((1, 4), dtype=torch.int32),
                                                       torch.zeros(1, dtype=torch.int32)),
@@ -42,6 +44,6 @@ def test_host_tensors_are_refused(name):
 
 def test_every_tensor_call_is_covered():
     tensor_calls = {"route", "route_threshold", "route_swap", "route_swap_blocks", "attention",
-                    "attention_counts", "uncertainty"}
+                    "attention_noalloc", "attention_counts", "uncertainty"}
     assert tensor_calls <= set(heta.__all__)
     assert tensor_calls == set(CALLS)

@@ -116,3 +116,23 @@ def test_noalloc_runs_unsplit_when_its_array_is_too_small(gpu_lib):
     err = np.abs(got - want)
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
     _against_oracle(w, q, k, v, dense.cpu().numpy(), got, 4096, 7)
+
+
+def test_binding_wrapper_matches_workspace_entry_point(gpu_lib):
+    """The Python binding's attention_noalloc passes its arguments to the same
+    entry point: bit for bit heta_attention's output where both plan the same
+    work."""
+    import torch
+    heta = gpu_lib
+    w = W.scaled(W.WAN21, H=2, d=128, grid=(8, 16, 24), win=(3, 9, 9), u_kind="uniform",
+                 u_seeds=(11,))
+    q, k, v = W.make_qkv(w)
+    Q, K, V = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+    kk = heta.dense_count(w.N, 0.2)
+    dense, _, _, _ = heta.route(to_dev(W.make_u(w)), kk)
+    want = from_dev_bf16(heta.attention(Q, K, V, w.grid, w.win, dense))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = from_dev_bf16(heta.attention_noalloc(Q, K, V, w.grid, w.win, dense, status=st))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert np.array_equal(got, want)

@@ -19,6 +19,7 @@ import os
 
 __all__ = ["load", "HetaError", "dense_count", "route", "route_threshold", "swap_count",
            "route_swap", "route_swap_blocks", "attention", "attention_counts",
+           "attention_noalloc",
            "attention_workspace_size", "attention_counts_workspace_size", "uncertainty",
            "selftest_wait_timeout", "status_string", "attention_flops", "LIB_PATH"]
 
@@ -82,6 +83,8 @@ def load():
     lib.heta_attention_counts_workspace_size.argtypes = ([i] * 10 +
                                                          [ctypes.POINTER(ctypes.c_size_t)])
     lib.heta_attention_counts_workspace_size.restype = i
+    lib.heta_attention_noalloc.argtypes = [vp, vp, vp] + [i] * 9 + [f, vp, i, vp, vp, vp]
+    lib.heta_attention_noalloc.restype = i
     _lib = lib
     return lib
 
@@ -296,6 +299,37 @@ def attention(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=Non
                                float(scale), pd if k > 0 else None, k, po, pw,
                                workspace.numel(), _opt(status), _stream())
     _check(rc, "heta_attention")
+    return out
+
+
+def attention_noalloc(Q, K, V, grid, win, dense_idx, *, scale=None, out=None, status=None):
+    """``attention`` without a workspace (``heta_attention_noalloc``): the
+    library's fixed device array serves as its scratch, so nothing is
+    allocated for the call (``out`` aside, when it is not passed).  Calls that
+    may overlap on the GPU race on that array; see include/heta.h."""
+    import torch
+    pq = _dev(Q, torch.bfloat16, "Q", 4)
+    pk = _dev(K, torch.bfloat16, "K", 4)
+    pv = _dev(V, torch.bfloat16, "V", 4)
+    if K.shape != Q.shape or V.shape != Q.shape:
+        raise ValueError("Q, K, V shapes differ")
+    B, H, N, d = Q.shape
+    Tg, Hg, Wg = grid
+    if Tg * Hg * Wg != N:
+        raise ValueError("grid %s does not hold N=%d tokens" % (grid, N))
+    pd = _dev(dense_idx, torch.int32, "dense_idx", 2)
+    if dense_idx.shape[0] != B:
+        raise ValueError("dense_idx batch mismatch")
+    k = dense_idx.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    po = _dev(out, torch.bfloat16, "out", 4)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = load().heta_attention_noalloc(pq, pk, pv, B, H, d, Tg, Hg, Wg, win[0], win[1], win[2],
+                                       float(scale), pd if k > 0 else None, k, po,
+                                       _opt(status), _stream())
+    _check(rc, "heta_attention_noalloc")
     return out
 
 
