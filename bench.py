@@ -614,6 +614,30 @@ def run_heta(args, info):
     # once all timing is done
     timed = (dense.cpu(), local.cpu(), out.cpu())
 
+    # ---- the same step captured once in a CUDA graph and replayed ---------------
+    graph = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        g_ms = e0.elapsed_time(e1) / args.steps
+        graph = {"ms_per_step": g_ms, "tokens_per_s": w.B * w.N / (g_ms / 1e3),
+                 "what": "route + attention + head captured once in a CUDA graph, replayed "
+                         "%d times (the timed line above launches them eagerly)" % args.steps}
+        del g
+    except Exception as e:  # noqa: BLE001 -- an extra measurement never fails the bench
+        graph = {"unavailable": "%s: %s" % (type(e).__name__, str(e)[:300])}
+    torch.cuda.synchronize()
+
     # ---- the same mask through PyTorch FlexAttention (comparison point) -------
     flex = None
     if not args.no_flex_compare and info.rank == 0:
@@ -883,6 +907,7 @@ def run_heta(args, info):
                           "peak": peaks["hbm_gbs"], "unit": "GB/s"},
         "dense_compare": dense_cmp,
         "flex_compare": flex,
+        "graph_replay": graph,
         "window_sweep": win_sweep,
         "other_configs": others,
         "threshold_mode": thr,
