@@ -373,8 +373,9 @@ def _time_ms(torch, fn, reps=5):
 
 
 def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
-    """The Wan2.2-5B shape, the batched two-sample step with the head, and the
-    rho sweep on uniform and clustered u at the Wan2.1 shape: CUDA-event times
+    """The Wan2.2-5B shape, the batched two-sample step with the head, the
+    Wan2.1 layer at 720p (21x45x80 = 75600 tokens), and the rho sweep on
+    uniform and clustered u at the Wan2.1 shape: CUDA-event times
     of the same calls as the main step (Q/K/V/X iid N(0,1) bf16 drawn on the
     device from a seeded generator; u from the workload's own generator)."""
     res = {}
@@ -408,7 +409,7 @@ def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
                 "attention_tflops": fl / (t_attn * 1e9),
                 "head_gbs": hbytes / (t_head * 1e6), "parity": par}
 
-    for w in (W.WAN22, W.BATCHED):
+    for w in (W.WAN22, W.BATCHED, W.WAN21_720P):
         Q, K, V = (randn_bf16(w.B, w.H, w.N, w.d) for _ in range(3))
         X = randn_bf16(w.B, w.N, w.C)
         wv = torch.from_numpy(W.make_head(W.scaled(w, B=1, grid=(1, 1, 8)))[1]).to(dev)
