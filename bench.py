@@ -419,7 +419,9 @@ def other_configs(heta, torch, dev, d_Q, d_K, d_V, out):
     sweep = {}
     q32, k32, v32 = bf16_host_f32(d_Q), bf16_host_f32(d_K), bf16_host_f32(d_V)
     for kind in ("uniform", "clustered"):
-        for rho in W.SWEEP_RHOS:
+        # uniform u also at the two ends: LOCAL items only (rho = 0) and
+        # DENSE items only (rho = 1)
+        for rho in W.SWEEP_RHOS + ((0.0, 1.0) if kind == "uniform" else ()):
             w = W.sweep(rho, kind)
             kk = heta.dense_count(w.N, rho)
             u_np = W.make_u(w)
