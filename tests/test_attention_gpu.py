@@ -234,3 +234,27 @@ def test_bad_dense_idx_is_reported_and_stays_in_bounds(gpu_lib, entry):
         want = oracle.attention(qf[b:b + 1], kf[b:b + 1], vf[b:b + 1], w.grid, w.win,
                                 keep[None, :])
         assert_close(got[b:b + 1].reshape(-1, d), want.reshape(-1, d), "sample %d" % b)
+
+
+def test_out_16_byte_aligned_gives_the_same_rows(gpu_lib):
+    """An out that is 16- but not 32-byte aligned takes the epilogue's
+    16-byte stores instead of its 32-byte ones; every row must equal, bit for
+    bit, the rows written into a 32-byte aligned out (DENSE and LOCAL rows
+    alike), and none may be left unwritten."""
+    import torch
+    heta = gpu_lib
+    w = MULTI_TILE[0]
+    q, k, v = W.make_qkv(w)
+    kk = heta.dense_count(w.N, 0.2)
+    Qd, Kd, Vd = to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v)
+    dense, _, _, _ = heta.route(to_dev(W.make_u(w)), kk)
+    a = torch.full_like(Qd, float("nan"))
+    buf = torch.full((Qd.numel() + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    b = buf[8:].view(Qd.shape)
+    assert a.data_ptr() % 32 == 0 and b.data_ptr() % 32 == 16
+    for out in (a, b):
+        heta.attention(Qd, Kd, Vd, w.grid, w.win, dense, out=out)
+    torch.cuda.synchronize()
+    ga, gb = from_dev_bf16(a), from_dev_bf16(b)
+    assert not np.isnan(ga).any(), "rows left unwritten"
+    assert np.array_equal(a.view(torch.int16).cpu().numpy(), b.view(torch.int16).cpu().numpy())

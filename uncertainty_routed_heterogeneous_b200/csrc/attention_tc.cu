@@ -67,6 +67,7 @@ constexpr uint32_t kItemConsumers = 1 + 256 + 32;
 struct Params {
     const uint16_t *Q;
     uint16_t *out;
+    int out32;        // out is 32-byte aligned (so is every row): 32-byte stores
     const int32_t *dense_idx;  // [B][k]
     const int32_t *k_dev;      // [B] dense rows per sample (<= k), or null: all k
     int32_t *status;
@@ -957,7 +958,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tmK3, const __grid_constant__
                     uint32_t o[32];
                     tmem_ld32(tO + 32 * c4, o);
                     tmem_wait_ld();
-                    if (store) {
+                    if (store && p.out32) {
+                        // 32-byte stores: each lane writes a whole sector of its row
+#pragma unroll
+                        for (int v = 0; v < 2; ++v) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                w[e] = pack_bf16(__uint_as_float(o[16 * v + 2 * e]) * inv,
+                                                 __uint_as_float(o[16 * v + 2 * e + 1]) * inv);
+                            st_global_v8(dst + c4 * 4 + 2 * v, w);
+                        }
+                    } else if (store) {
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             uint4 w;
@@ -1159,6 +1171,7 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &pl, void *worksp
     Params p;
     p.Q = a.Q;
     p.out = a.out;
+    p.out32 = (reinterpret_cast<uintptr_t>(a.out) & 31u) == 0;
     p.dense_idx = a.dense_idx;
     p.k_dev = a.k_dev;
     p.status = a.status;
