@@ -228,7 +228,9 @@ HETA_API heta_status heta_attention_workspace_size(int B, int H, int d, int Tg, 
  *              its dense result, its local result or no write), but every
  *              read stays inside Q, K, V and dense_idx and every write inside
  *              out.
- *   out        [B,H,N,d] bf16 out; every row is written exactly once.
+ *   out        [B,H,N,d] bf16 out; every row is written exactly once.  A
+ *              32-byte aligned out (any fresh allocation) is written 32 bytes
+ *              a store, a 16-byte aligned one 16 bytes a store (same values).
  *   scale      softmax scale, normally 1/sqrt(d).
  *   workspace  device scratch of at least heta_attention_workspace_size()
  *              bytes, 16-byte aligned, owned by the caller; its contents on
