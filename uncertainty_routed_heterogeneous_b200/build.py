@@ -6,7 +6,9 @@ Each ``csrc/*.cu`` is compiled to an object under ``_build/`` (in parallel),
 then linked into ``uncertainty_routed_heterogeneous_b200/libheta.so``.  nvcc
 cross-compiles without a GPU.  The CUDA runtime is linked statically and the
 driver entry point for tensor-map encoding is fetched at run time, so the
-library needs no libcuda at link time.
+library needs no libcuda at link time.  The plain-C example
+``examples/heta_run.c`` (the path driven through ``include/heta.h`` alone) is
+built next to it as ``examples/heta_run``.
 """
 import concurrent.futures as cf
 import glob
@@ -20,6 +22,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libheta.so")
+EXAMPLE_SRC = os.path.join(PKG, "examples", "heta_run.c")
+EXAMPLE = os.path.join(PKG, "examples", "heta_run")
+CUDA_HOME = os.environ.get("CUDA_HOME", "/usr/local/cuda")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -75,7 +80,24 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
         if r.returncode != 0:
             raise RuntimeError("link failed:\n%s\n%s" % (r.stdout, r.stderr))
         os.replace(tmp, LIB)
+    build_example(force)
     return LIB
+
+
+def build_example(force: bool = False) -> str:
+    """gcc-compiles examples/heta_run.c against include/heta.h, libheta.so and
+    the CUDA runtime (for its allocations and copies); returns its path."""
+    if force or _stale(EXAMPLE, [EXAMPLE_SRC, LIB] + glob.glob(os.path.join(INCLUDE, "*.h"))):
+        tmp = EXAMPLE + ".tmp.%d" % os.getpid()
+        cmd = [os.environ.get("CC", "gcc"), "-std=c11", "-O2", "-Wall", "-Wextra", "-Werror",
+               "-I", INCLUDE, "-I", os.path.join(CUDA_HOME, "include"), EXAMPLE_SRC, "-o", tmp,
+               "-L", PKG, "-lheta", "-L", os.path.join(CUDA_HOME, "lib64"), "-lcudart", "-lm",
+               "-Wl,-rpath,$ORIGIN/..", "-Wl,-rpath," + os.path.join(CUDA_HOME, "lib64")]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError("the C example failed to build:\n%s\n%s" % (r.stdout, r.stderr))
+        os.replace(tmp, EXAMPLE)
+    return EXAMPLE
 
 
 if __name__ == "__main__":
