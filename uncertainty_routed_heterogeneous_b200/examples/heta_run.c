@@ -111,6 +111,10 @@ int main(int argc, char **argv)
             return 1;
         }
     }
+    if ((int64_t)Tg * Hg * Wg > INT32_MAX) {
+        fprintf(stderr, "heta_run: the grid holds more than 2^31 - 1 tokens\n");
+        return 1;
+    }
     const int N = Tg * Hg * Wg;
     const size_t qkv_bytes = (size_t)B * H * N * d * 2;
     const size_t u_bytes = (size_t)B * N * 4;
